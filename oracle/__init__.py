@@ -1,0 +1,7 @@
+"""FP64 CPU oracle for paged decode attention (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  The product path (the CUDA library and its
+binding) never does.
+"""
+from .oracle import append, gather, decode, OracleError  # noqa: F401

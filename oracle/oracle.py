@@ -1,0 +1,109 @@
+"""ctypes wrapper around libpkv_oracle.so (TEST INFRASTRUCTURE ONLY).
+
+Arrays are numpy: the pool is uint16 [num_pages, 2, 8, 16, 64] (BF16 bits,
+layout page[kv][kv_head][slot][d]); block tables int32
+[num_layers, batch, max_blocks]; seq_lens int32 [batch] (length after the
+step's append); q uint16 [batch, 32, 64]; k_new / v_new uint16 [batch, 8, 64].
+Outputs of decode are float64 [batch, 32, 64].
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+_CODES = {1: "bad argument", 2: "bad sequence length", 3: "block-table entry outside the pool"}
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code):
+        super().__init__("oracle: %s (code %d)" % (_CODES.get(code, "?"), code))
+        self.code = code
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i32 = ctypes.c_int32
+        lib.pkvo_append.argtypes = [P, i32, P, i32, i32, i32, P, P, P, i32]
+        lib.pkvo_gather.argtypes = [P, i32, P, i32, i32, i32, P, i32, P, P, i32]
+        lib.pkvo_decode.argtypes = [P, P, i32, P, i32, i32, i32, P, i32, ctypes.c_double,
+                                    P, P, i32, i32]
+        for f in (lib.pkvo_append, lib.pkvo_gather, lib.pkvo_decode):
+            f.restype = ctypes.c_int
+        _LIB = lib
+    return _LIB
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError("expected %s, got %s" % (np.dtype(dtype), a.dtype))
+    return a
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc):
+    if rc != 0:
+        raise OracleError(rc)
+
+
+def append(pool, block_tables, seq_lens, k_new, v_new, layer):
+    """In-place append of one token per sequence (see pkv_oracle.h)."""
+    if not (pool.flags.c_contiguous and pool.dtype == np.uint16):
+        raise TypeError("pool must be C-contiguous uint16")
+    bt = _c(block_tables, np.int32)
+    sl = _c(seq_lens, np.int32)
+    k = _c(k_new, np.uint16)
+    v = _c(v_new, np.uint16)
+    L, B, MB = bt.shape
+    _check(_lib().pkvo_append(_p(pool), pool.shape[0], _p(bt), L, B, MB, _p(sl), _p(k), _p(v),
+                              int(layer)))
+
+
+def gather(pool, block_tables, seq_lens, layer, max_seq_len, k_out=None, v_out=None):
+    """Contiguous copy-out of K and V, [batch, 8, max_seq_len, 64] uint16 each."""
+    pool = _c(pool, np.uint16)
+    bt = _c(block_tables, np.int32)
+    sl = _c(seq_lens, np.int32)
+    L, B, MB = bt.shape
+    if k_out is None:
+        k_out = np.zeros((B, 8, max_seq_len, 64), np.uint16)
+    if v_out is None:
+        v_out = np.zeros((B, 8, max_seq_len, 64), np.uint16)
+    _check(_lib().pkvo_gather(_p(pool), pool.shape[0], _p(bt), L, B, MB, _p(sl), int(layer),
+                              _p(k_out), _p(v_out), int(max_seq_len)))
+    return k_out, v_out
+
+
+def decode(q, pool, block_tables, seq_lens, layer, scale, rows=None, nthreads=None, out=None):
+    """FP64 decode attention; returns float64 [batch, 32, 64].
+
+    rows: optional list of sequence indices to compute (others stay as in
+    ``out``, zeros by default).  nthreads: worker threads (default: all cores).
+    """
+    q = _c(q, np.uint16)
+    pool = _c(pool, np.uint16)
+    bt = _c(block_tables, np.int32)
+    sl = _c(seq_lens, np.int32)
+    L, B, MB = bt.shape
+    if out is None:
+        out = np.zeros((B, 32, 64), np.float64)
+    if rows is None:
+        rp, nr = None, B
+    else:
+        rows_a = _c(np.asarray(rows, np.int32), np.int32)
+        rp, nr = _p(rows_a), rows_a.size
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    _check(_lib().pkvo_decode(_p(q), _p(pool), pool.shape[0], _p(bt), L, B, MB, _p(sl),
+                              int(layer), float(scale), _p(out), rp, nr, int(nthreads)))
+    return out

@@ -1,0 +1,69 @@
+"""Small random paged-cache cases for tests (numpy RNG, seeded).
+
+Builds a pool with a random physical placement of every sequence's pages,
+NaN in every slot that holds no token, and random N(0,1) BF16 values
+elsewhere.  Holds no attention arithmetic.
+"""
+import numpy as np
+
+T, G, H, D = 16, 8, 32, 64
+NAN = 0x7FC0
+
+
+def bf16_bits(x):
+    """float array -> BF16 bit patterns, round to nearest even."""
+    f = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    rnd = ((f >> 16) & 1) + 0x7FFF
+    return ((f + rnd) >> 16).astype(np.uint16)
+
+
+def bf16_to_f64(b):
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def make_case(lens, seed=0, num_layers=1, spare_pages=3, max_blocks=None):
+    """lens: lengths after the append (decode attends to all of them).
+    Returns dict(pool, bt, seq_lens, q, k_new, v_new) with the new token's
+    K/V already stored in the pool and also returned as k_new / v_new."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, np.int32)
+    B = lens.size
+    need = [(int(l) + T - 1) // T for l in lens]
+    mb = max(1, max(need)) if max_blocks is None else max_blocks
+    n_pages = num_layers * sum(need) + spare_pages
+    perm = rng.permutation(n_pages).astype(np.int32)
+    bt = np.full((num_layers, B, mb), -1, np.int32)
+    cur = 0
+    for l in range(num_layers):
+        for b in range(B):
+            bt[l, b, :need[b]] = perm[cur:cur + need[b]]
+            cur += need[b]
+    pool = np.full((n_pages, 2, G, T, D), NAN, np.uint16)
+    for l in range(num_layers):
+        for b in range(B):
+            for t in range(int(lens[b])):
+                p = bt[l, b, t // T]
+                pool[p, :, :, t % T, :] = bf16_bits(rng.standard_normal((2, G, D)))
+    q = bf16_bits(rng.standard_normal((B, H, D)))
+    k_new = np.zeros((B, G, D), np.uint16)
+    v_new = np.zeros((B, G, D), np.uint16)
+    for b in range(B):
+        if lens[b] > 0:
+            t = int(lens[b]) - 1
+            p = bt[0, b, t // T]
+            k_new[b] = pool[p, 0, :, t % T, :]
+            v_new[b] = pool[p, 1, :, t % T, :]
+    return dict(pool=pool, bt=bt, seq_lens=lens, q=q, k_new=k_new, v_new=v_new)
+
+
+def contiguous_kv(case, layer=0):
+    """Numpy fancy-index gather of K and V per sequence: list of
+    (K [G, L, D], V [G, L, D]) float64 arrays."""
+    out = []
+    for b, L in enumerate(case["seq_lens"]):
+        t = np.arange(int(L))
+        pages = case["bt"][layer, b, t // T]
+        K = case["pool"][pages, 0, :, t % T, :]   # [L, G, D]
+        V = case["pool"][pages, 1, :, t % T, :]
+        out.append((bf16_to_f64(K).transpose(1, 0, 2), bf16_to_f64(V).transpose(1, 0, 2)))
+    return out
