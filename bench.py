@@ -1,0 +1,409 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged decode-attention hot path on B200.
+
+One step = one decode step of the whole model's attention cache traffic:
+for each of the 16 layers, append the new token's K/V of every sequence
+(pkv_append) and run decode attention over the paged cache
+(paged_attention_decode), through the C ABI.  Default workload: the
+continuous-batching mix (batch 64, lengths log-uniform in [1, 8192],
+fragmented block tables, 16 layers).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--kernel auto|simt|mma]
+
+Prints one JSON line (rank 0).  ``value`` is decode-queries/s over all
+ranks, one query being one sequence's 32 query heads at one layer.  The
+``roofline`` object reports the decode kernel's algorithmic HBM bytes per
+launch divided by its measured average launch time, against the measured
+HBM copy bandwidth.  ``--impl reference`` times the FP64 CPU oracle on the
+same workload instead (bounded sample per step, host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_attention_decode_pkv_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention: achieved HBM GB/s (% of peak) and decode-queries/sec"
+UNIT = "decode-queries/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ helpers --
+
+def alg_bytes_decode(seq_lens: np.ndarray) -> int:
+    """Algorithmic bytes of one decode launch: per sequence K+V of every
+    token (2048 B/token), q (4096 B), FP32 out (8192 B), block-table entries
+    (4 B per page) and the length (4 B)."""
+    L = seq_lens.astype(np.int64)
+    return int((2048 * L + 4096 + 8192 + 4 * ((L + 15) // 16) + 4).sum())
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons, taken while the
+    timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm --
+
+class Runner:
+    """Device-resident state of one workload on one GPU."""
+
+    def __init__(self, w: W.Workload, device, kernel: int):
+        from paged_attention_decode_pkv_b200 import pkv
+        self.pkv = pkv
+        self.w = w
+        self.device = device
+        self.kernel = kernel
+        self.pool_t = W.make_pool(w, device)
+        self.pool = pkv.Pool(w.num_pages, storage=self.pool_t)
+        self.bt = torch.from_numpy(w.block_tables).to(device)
+        nl, B = w.num_layers, w.batch
+        self.seq_lens = [torch.from_numpy(w.seq_lens(s)).to(device)
+                         for s in range(1, w.num_steps + 1)]
+        # one set of per-layer inputs, reused every step (values do not change timing)
+        ins = [W.step_inputs(w, 1, l, device) for l in range(nl)]
+        self.q = torch.stack([x[0] for x in ins])
+        self.k = torch.stack([x[1] for x in ins])
+        self.v = torch.stack([x[2] for x in ins])
+        self.out = torch.empty((nl, B, 32, 64), dtype=torch.float32, device=device)
+        self.ws = self.pool.workspace(B, kernel)
+        self.step_idx = 0
+
+    def step(self, stream, ev_pairs=None):
+        """One decode step over all layers; optionally records (start, end)
+        events around every decode launch."""
+        pkv = self.pkv
+        sl = self.seq_lens[self.step_idx % self.w.num_steps]
+        self.step_idx += 1
+        for l in range(self.w.num_layers):
+            pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
+            if ev_pairs is not None:
+                e0, e1 = ev_pairs.pop()
+                e0.record(stream)
+            pkv.decode(self.q[l], self.pool, self.bt, sl, l, self.w.scale, out=self.out[l],
+                       workspace=self.ws, kernel=self.kernel, stream=stream)
+            if ev_pairs is not None:
+                e1.record(stream)
+                self.used.append((e0, e1))
+
+    def step_bytes(self, step_idx):
+        sl = self.w.seq_lens(step_idx % self.w.num_steps + 1)
+        return alg_bytes_decode(sl)
+
+
+def run_ours(args, rank, world, local_rank):
+    from paged_attention_decode_pkv_b200 import pkv
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    kernel = {"auto": pkv.KERNEL_AUTO, "simt": pkv.KERNEL_SIMT, "mma": pkv.KERNEL_MMA}[args.kernel]
+    w = W.make(args.workload, seed=W.make(args.workload).seed + 1000 * rank) if rank else \
+        W.make(args.workload)
+    r = Runner(w, device, kernel)
+    stream = torch.cuda.Stream(device)
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            r.step(stream)
+    stream.synchronize()
+    assert pkv.get_device_error(r.pool, stream) == 0
+
+    # ---- timed region: K steps, decode launches bracketed by events
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps * w.num_layers)]
+    r.used = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    first_step = r.step_idx
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(args.steps):
+                r.step(stream, pairs)
+            t1.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in r.used]
+    dec_bytes = [r.step_bytes(first_step + i // w.num_layers) for i in range(len(dec_ms))]
+    err = pkv.get_device_error(r.pool, stream)
+    if err != 0:
+        raise RuntimeError("device error during timed region: %s" % pkv.status_string(err))
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+    queries = args.steps * w.num_layers * w.batch * world
+    value = queries / (ms / 1e3)
+
+    # ---- end to end through the public API from pinned host buffers
+    e2e = run_e2e(r, stream, min(args.steps, args.e2e_steps), barrier, dist, device)
+
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peaks()
+    avg_dec_s = sum(dec_ms) / len(dec_ms) / 1e3
+    avg_bytes = sum(dec_bytes) / len(dec_bytes)
+    achieved = avg_bytes / avg_dec_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": w.name, "description": w.description, "batch": w.batch,
+            "layers": w.num_layers, "pool_pages": w.num_pages,
+            "kv_bytes_per_layer": w.kv_bytes(1), "accumulate": "f32",
+            "kernel": args.kernel, "parallelism": "dp%d (independent replicas)" % world,
+            "l2": "inputs larger than L2: one step reads %.0f MB of K/V" %
+                  (w.kv_bytes(1) * w.num_layers / 1e6),
+        },
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+            "kernel": "decode_kernel", "alg_bytes_per_launch": avg_bytes,
+            "avg_launch_us": avg_dec_s * 1e6, "launches": len(dec_ms),
+        },
+        "decode_only_queries_per_s": w.batch / avg_dec_s,
+        "e2e": e2e,
+        "gpu_launches": args.steps * w.num_layers * 2,
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, r.pool_t, args.cpu_seconds)
+    return line
+
+
+def run_e2e(r: Runner, stream, steps, barrier, dist, device):
+    """Same step, with every step's inputs (q, k_new, v_new of all layers,
+    seq_lens) copied from pinned host memory and all outputs copied back."""
+    w = r.w
+    hq = r.q.cpu().pin_memory()
+    hk = r.k.cpu().pin_memory()
+    hv = r.v.cpu().pin_memory()
+    hsl = [x.cpu().pin_memory() for x in r.seq_lens]
+    hout = torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory()
+    sl_dev = torch.empty_like(r.seq_lens[0])
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + hsl[0].numel() * 4
+    d2h = hout.numel() * 4
+    pkv = r.pkv
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(steps):
+            r.q.copy_(hq, non_blocking=True)
+            r.k.copy_(hk, non_blocking=True)
+            r.v.copy_(hv, non_blocking=True)
+            sl_dev.copy_(hsl[i % w.num_steps], non_blocking=True)
+            for l in range(w.num_layers):
+                pkv.append(r.pool, r.bt, sl_dev, r.k[l], r.v[l], l, stream=stream)
+                pkv.decode(r.q[l], r.pool, r.bt, sl_dev, l, w.scale, out=r.out[l],
+                           workspace=r.ws, kernel=r.kernel, stream=stream)
+            hout.copy_(r.out, non_blocking=True)
+        t1.record(stream)
+    stream.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    if dist:
+        import torch.distributed as tdist
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+    world = tdist_world() if dist else 1
+    return {"value": steps * w.num_layers * w.batch * world / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+def tdist_world():
+    import torch.distributed as tdist
+    return tdist.get_world_size()
+
+
+# ------------------------------------------------------------ oracle arms --
+
+def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None):
+    """Time the FP64 oracle on whole-layer decodes of step 1 (all sequences
+    of the batch), layer after layer, until ``max_seconds`` have passed.
+    Returns (queries, seconds, threads, layers_done)."""
+    import oracle
+    layers = list(range(w.num_layers)) if layers is None else layers
+    threads = os.cpu_count() or 1
+    sl = w.seq_lens(1)
+    done, secs = 0, 0.0
+    for l in layers:
+        pool_h, bt_h = W.compact_pages(w, pool_t, range(w.batch), [l])
+        q, k, v = W.step_inputs(w, 1, l, pool_t.device)
+        qb, kb, vb = W.bits(q), W.bits(k), W.bits(v)
+        t = time.perf_counter()
+        oracle.append(pool_h, bt_h, sl, kb, vb, l)
+        oracle.decode(qb, pool_h, bt_h, sl, l, w.scale, nthreads=threads)
+        secs += time.perf_counter() - t
+        done += 1
+        if secs >= max_seconds:
+            break
+    return done * w.batch, secs, threads, done
+
+
+def cpu_baseline(w, pool_t, max_seconds):
+    q, s, thr, layers = oracle_sample(w, pool_t, max_seconds)
+    return {"value": q / s, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": "%d whole-layer append+decode(s) of step 1 (%d sequences each), "
+                      "%.1f s of FP64 oracle work" % (layers, w.batch, s)}
+
+
+def run_reference(args, rank, world, local_rank):
+    """The oracle as the reference arm: each step is a bounded sample (one
+    whole-layer append + decode of all sequences) of the same workload."""
+    if rank != 0:
+        return None
+    w = W.make(args.workload)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    if W.Workload.pool_bytes(w) > 8e9 and dev == "cpu":
+        raise SystemExit("pool too large to generate on the host")
+    pool_t = W.make_pool(w, dev)
+    nl = w.num_layers
+    for i in range(args.warmup):
+        oracle_sample(w, pool_t, 0.0, layers=[i % nl])
+    q_tot, s_tot = 0, 0.0
+    thr = 1
+    for i in range(args.steps):
+        q, s, thr, _ = oracle_sample(w, pool_t, 0.0, layers=[i % nl])
+        q_tot += q
+        s_tot += s
+    v = q_tot / s_tot
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_tot / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "description": w.description, "batch": w.batch,
+                   "layers": nl, "sample": "one whole-layer append+decode per step"},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": "%d steps x one layer of %d sequences" % (args.steps, w.batch)},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# --------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="continuous_batching_b64", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "mma"])
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world, local_rank)
+        else:
+            line = run_ours(args, rank, world, local_rank)
+        if line is not None and rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * pkv.h -- C ABI of libpkv: paged KV-cache decode attention for B200 (sm_100a).
+ *
+ * The method (sources, by page title and section):
+ *  - "Curso gratuito recorre la inferencia de LLM con videos, notas y un
+ *    motor funcional en C++", section "¿Cómo administra el motor la memoria
+ *    de la caché KV?": one shared pool of BF16 pages, each physical page
+ *    holding the keys and values of 16 tokens, a block table per sequence
+ *    and layer, and decode attention that reads each sequence's pages in
+ *    place with an FP32 online softmax instead of gathering a contiguous
+ *    prefix.
+ *  - comrad404 article on samir-vllm ("Как устроен путь от текста запроса
+ *    до следующего токена в языковой модели?"), section "Что README говорит
+ *    о KV-кэше и пакетном декодировании": each decode step adds the new
+ *    token's K/V to the cache.
+ *  - "Construye tu propio motor de inferencia LLM de alto rendimiento en C++
+ *    y CUDA", sections "La arquitectura del modelo: Llama 3.2 1B" (32 query
+ *    heads, 8 kv heads, head dimension 64) and "Atención de Consulta
+ *    Agrupada (GQA)" (query head h reads kv head h / 4).
+ *
+ * Conventions shared by every call:
+ *  - Every call returns an int status (pkv_status).  No call aborts, exits
+ *    or traps.  Host-visible argument errors are returned at once and
+ *    nothing is launched.
+ *  - Every device pointer is caller-owned device memory (for instance a
+ *    torch tensor's data_ptr()).  The library keeps no pointer to it after
+ *    the call returns.
+ *  - Every kernel call is asynchronous on the given stream and allocates
+ *    nothing.  A NULL stream is the legacy default stream.
+ *  - Errors that only the device can see (a block-table entry outside the
+ *    pool, a sequence length out of range, a timed-out wait) never fault:
+ *    the kernel skips the offending work, leaves the result for that
+ *    sequence unspecified, and records the first such error in a sticky
+ *    word of the pool, read and cleared by pkv_get_device_error().
+ *  - BF16 values are passed as their 16-bit patterns (uint16_t).
+ *
+ * Layouts (the pages fix none of them; these are this library's readings):
+ *  - Pool page p (32768 bytes) = [kv in {K=0, V=1}][kv head g < 8]
+ *    [slot s < 16][d < 64] BF16, so element (p, kv, g, s, d) sits at
+ *    ((((p*2 + kv)*8 + g)*16 + s)*64 + d) * 2 bytes from the pool base.
+ *    Token t of a sequence lives in slot t % 16 of logical page t / 16.
+ *  - Block tables: int32 [num_layers][batch][max_blocks], row-major;
+ *    entry [layer][b][j] is the physical page of logical page j of
+ *    sequence b at that layer.  Entries past a sequence's last page are
+ *    never read.
+ *  - seq_lens: int32 [batch], the context length AFTER this step's append.
+ *    The new token sits at position L-1; decode attends to 0..L-1.
+ *  - q: BF16 [batch][32][64]; k_new, v_new: BF16 [batch][8][64];
+ *    out: FP32 [batch][32][64].
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#define PKV_PAGE_TOKENS 16
+#define PKV_NUM_KV_HEADS 8
+#define PKV_NUM_Q_HEADS 32
+#define PKV_HEAD_DIM 64
+#define PKV_PAGE_BYTES 32768
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *pkv_stream_t;
+
+/* Opaque pool handle; owned by the caller between create and destroy. */
+typedef struct pkv_pool pkv_pool;
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = -1,    /* null pointer, negative size, layer out of range  */
+  PKV_ERR_UNSUPPORTED = -2,    /* shape other than 16 tokens / 8 kv heads / d 64    */
+  PKV_ERR_CUDA = -3,           /* a CUDA runtime call failed                        */
+  PKV_ERR_OUT_OF_PAGES = -4,   /* reserved for page allocators built on this ABI    */
+  PKV_ERR_BAD_PAGE = -5,       /* device: block-table entry outside [0, num_pages)  */
+  PKV_ERR_WORKSPACE = -6,      /* workspace missing, misaligned or too small        */
+  PKV_ERR_DEVICE_TIMEOUT = -7, /* device: a bounded wait on a copy ran out           */
+  PKV_ERR_BAD_SEQ_LEN = -8     /* device: seq_len < 0 (append: < 1) or too long      */
+} pkv_status;
+
+/* Decode kernel variants for paged_attention_decode_ex. */
+#define PKV_KERNEL_AUTO 0
+#define PKV_KERNEL_SIMT 1 /* CUDA-core FP32 dot products, warp-shuffle reductions */
+#define PKV_KERNEL_MMA 2  /* tensor-core (mma.sync BF16) QK and PV, FP32 softmax   */
+
+/*
+ * Create a pool of num_pages pages on the current CUDA device.
+ * page_tokens, num_kv_heads and head_dim must be 16, 8 and 64 (else
+ * PKV_ERR_UNSUPPORTED).  device_storage: caller-owned device memory of at
+ * least num_pages * PKV_PAGE_BYTES bytes (storage_bytes), 16-byte aligned;
+ * or NULL, in which case the library allocates (and later frees) it.  The
+ * pool's contents are not initialised.  Also allocates a 4-byte device
+ * error word.  The pages' engine sizes its pool with a command-line flag
+ * (128 MiB by default), which is what num_pages expresses here.
+ */
+PKV_API int pkv_pool_create(int32_t num_pages, int32_t page_tokens, int32_t num_kv_heads,
+                    int32_t head_dim, void *device_storage, size_t storage_bytes,
+                    pkv_pool **out);
+
+/* Free the pool handle and whatever the library allocated for it (not
+ * caller-owned storage).  Synchronises the device. NULL is accepted. */
+PKV_API int pkv_pool_destroy(pkv_pool *pool);
+
+/* Device pointer to page 0 of the pool (layout above), or NULL. */
+PKV_API void *pkv_pool_data(const pkv_pool *pool);
+
+/* Number of pages, or -1 for a NULL pool. */
+PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
+
+/*
+ * Append (decode step, one token per sequence): for each b with
+ * L = seq_lens[b], copy k_new[b][g][:] and v_new[b][g][:] for all 8 kv
+ * heads into slot (L-1) % 16 of page block_tables[layer][b][(L-1)/16].
+ * Bit copies.  seq_lens is not modified (the caller advances it).  Two
+ * sequences appending into the same page slot is undefined.  Device errors:
+ * L < 1 or L > max_blocks*16 -> PKV_ERR_BAD_SEQ_LEN, page outside the pool
+ * -> PKV_ERR_BAD_PAGE; that sequence is skipped.
+ */
+PKV_API int pkv_append(pkv_pool *pool, const int32_t *block_tables, const int32_t *seq_lens,
+               const uint16_t *k_new, const uint16_t *v_new, int32_t layer,
+               int32_t num_layers, int32_t batch, int32_t max_blocks, pkv_stream_t stream);
+
+/*
+ * Workspace bytes paged_attention_decode needs for this batch on the pool's
+ * device (split-KV partial results and merge counters).  The workspace is
+ * caller-owned device memory, 256-byte aligned, and must be ZERO-FILLED
+ * before its first use.  Every decode that completes puts the part that must
+ * start at zero (one merge counter per (sequence, kv head)) back to zero, so
+ * the workspace can be reused without clearing it; after a
+ * PKV_ERR_DEVICE_TIMEOUT zero it again.  Calls that share one workspace must
+ * not overlap in time.
+ */
+PKV_API int pkv_decode_workspace_bytes(const pkv_pool *pool, int32_t batch, size_t *bytes_out);
+
+/*
+ * Decode attention of one new query token per sequence at one layer:
+ *   out[b][h][:] = sum_{t<L} softmax_t(scale * q[b][h].K[t][h/4]) V[t][h/4]
+ * with K/V read in place from the pages block_tables[layer][b][*], FP32
+ * online softmax and FP32 accumulation.  Sequences with L == 0 get an
+ * all-zero output.  Long contexts are split across the GPU (split-KV) and
+ * merged with log-sum-exp weights inside the same launch.  Device errors:
+ * L < 0 or L > max_blocks*16 -> PKV_ERR_BAD_SEQ_LEN (that row is written as
+ * zeros); a page outside the pool -> PKV_ERR_BAD_PAGE (that page is
+ * skipped).  Requires 8 * batch * max_blocks < 2^31.
+ */
+PKV_API int paged_attention_decode(const uint16_t *q, const pkv_pool *pool, const int32_t *block_tables,
+                           const int32_t *seq_lens, int32_t layer, float scale, float *out,
+                           int32_t num_layers, int32_t batch, int32_t max_blocks,
+                           void *workspace, size_t workspace_bytes, pkv_stream_t stream);
+
+/*
+ * As paged_attention_decode, with tuning/testing knobs:
+ *   kernel:      PKV_KERNEL_AUTO / _SIMT / _MMA;
+ *   grid_ctas:   0 = one persistent wave over the device; > 0 = exactly that
+ *                many CTAs (the split of long contexts changes with it; the
+ *                workspace needed is pkv_decode_workspace_bytes_ex's);
+ *   min_chunk:   0 = automatic; > 0 = each warp takes at least this many
+ *                (page, kv-head) tiles.
+ */
+PKV_API int paged_attention_decode_ex(const uint16_t *q, const pkv_pool *pool,
+                              const int32_t *block_tables, const int32_t *seq_lens, int32_t layer,
+                              float scale, float *out, int32_t num_layers, int32_t batch,
+                              int32_t max_blocks, void *workspace, size_t workspace_bytes,
+                              pkv_stream_t stream, int32_t kernel, int32_t grid_ctas,
+                              int32_t min_chunk);
+
+/* Workspace bytes for paged_attention_decode_ex with these knobs. */
+PKV_API int pkv_decode_workspace_bytes_ex(const pkv_pool *pool, int32_t batch, int32_t kernel,
+                                  int32_t grid_ctas, size_t *bytes_out);
+
+/*
+ * Gather (page indexing made visible): k_out[b][g][t][:] and v_out[b][g][t][:]
+ * = K and V of token t of sequence b at `layer`, for t < seq_lens[b]; rows
+ * t >= seq_lens[b] are not written.  k_out, v_out: BF16 [batch][8]
+ * [max_seq_len][64].  Device errors: L < 0, L > max_seq_len or
+ * L > max_blocks*16 -> PKV_ERR_BAD_SEQ_LEN; page outside the pool ->
+ * PKV_ERR_BAD_PAGE (those rows are not written).
+ */
+PKV_API int pkv_gather(const pkv_pool *pool, const int32_t *block_tables, const int32_t *seq_lens,
+               int32_t layer, uint16_t *k_out, uint16_t *v_out, int32_t num_layers,
+               int32_t batch, int32_t max_blocks, int32_t max_seq_len, pkv_stream_t stream);
+
+/* Synchronise `stream`, return in *status_out the first device error
+ * recorded since the last call (PKV_OK if none) and clear it. */
+PKV_API int pkv_get_device_error(pkv_pool *pool, pkv_stream_t stream, int32_t *status_out);
+
+/* Static English text for a status code. */
+PKV_API const char *pkv_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

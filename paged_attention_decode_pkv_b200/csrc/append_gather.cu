@@ -1,0 +1,112 @@
+// append_gather.cu -- KV-append scatter and block-table page gather.
+//
+// Append: each decode step adds the new token's K/V to the cache (comrad404
+// article on samir-vllm, section "Что README говорит о KV-кэше и пакетном
+// декодировании"); the token goes to slot (L-1) % 16 of the page that the
+// sequence's block table names for logical page (L-1) / 16 ("Curso gratuito
+// recorre la inferencia de LLM...", section on the KV cache).
+//
+// Gather: the same block-table walk, copying a sequence's tokens out into a
+// contiguous [8][max_seq_len][64] layout.  Decode never does this (it reads
+// pages in place); the gather exists so that page indexing can be checked
+// bit for bit.
+//
+// Both are pure 16-byte copies: 8 consecutive threads move one 128-byte row
+// (one token of one kv head), so every warp access is four full 128-byte
+// lines.
+#include "pkv_internal.cuh"
+
+namespace pkv {
+
+// One CTA per sequence, 128 threads = (K|V) x 8 kv heads x 8 chunks of 16 B.
+__global__ void __launch_bounds__(128) append_kernel(const uint4* __restrict__ k_new,
+                                                     const uint4* __restrict__ v_new,
+                                                     uint4* __restrict__ pool,
+                                                     const int32_t* __restrict__ bt,
+                                                     const int32_t* __restrict__ seq_lens,
+                                                     int32_t* __restrict__ err, int32_t max_blocks,
+                                                     int32_t num_pages) {
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int kv = tid >> 6;
+  const int g = (tid >> 3) & 7;
+  const int c = tid & 7;
+  const int32_t L = seq_lens[b];
+  if (L < 1 || static_cast<int64_t>(L) > static_cast<int64_t>(max_blocks) * kTokens) {
+    if (tid == 0) record_error(err, kErrBadLen);
+    return;
+  }
+  const int32_t pos = L - 1;
+  const int32_t phys = bt[static_cast<int64_t>(b) * max_blocks + pos / kTokens];
+  if (phys < 0 || phys >= num_pages) {
+    if (tid == 0) record_error(err, kErrBadPage);
+    return;
+  }
+  const int slot = pos % kTokens;
+  // source: [B][8][64] BF16 = 8 chunks of 16 B per (b, g)
+  const uint4* src = (kv ? v_new : k_new) + (static_cast<int64_t>(b) * kKvHeads + g) * 8 + c;
+  // destination row (phys, kv, g, slot): 128 B = 8 chunks
+  const int64_t row = (static_cast<int64_t>(phys) * 2 + kv) * (kKvHeads * kTokens) +
+                      g * kTokens + slot;
+  pool[row * 8 + c] = *src;
+}
+
+// grid (ceil(max_seq_len / 32), 8 kv heads, batch); 256 threads = 32 tokens
+// x 8 chunks of 16 B; each thread copies one K chunk and one V chunk.
+__global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ pool,
+                                                     const int32_t* __restrict__ bt,
+                                                     const int32_t* __restrict__ seq_lens,
+                                                     uint4* __restrict__ k_out,
+                                                     uint4* __restrict__ v_out,
+                                                     int32_t* __restrict__ err, int32_t max_blocks,
+                                                     int32_t num_pages, int32_t max_seq_len) {
+  const int b = blockIdx.z;
+  const int g = blockIdx.y;
+  const int t = blockIdx.x * 32 + (threadIdx.x >> 3);
+  const int c = threadIdx.x & 7;
+  const int32_t L = seq_lens[b];
+  if (L < 0 || L > max_seq_len ||
+      static_cast<int64_t>(L) > static_cast<int64_t>(max_blocks) * kTokens) {
+    if (blockIdx.x == 0 && g == 0 && threadIdx.x == 0) record_error(err, kErrBadLen);
+    return;
+  }
+  if (t >= L) return;
+  const int32_t phys = bt[static_cast<int64_t>(b) * max_blocks + t / kTokens];
+  if (phys < 0 || phys >= num_pages) {
+    if ((t % kTokens) == 0 && c == 0) record_error(err, kErrBadPage);
+    return;
+  }
+  const int64_t krow = (static_cast<int64_t>(phys) * 2) * (kKvHeads * kTokens) + g * kTokens +
+                       (t % kTokens);
+  const int64_t vrow = krow + kKvHeads * kTokens;
+  const int64_t orow = (static_cast<int64_t>(b) * kKvHeads + g) * max_seq_len + t;
+  k_out[orow * 8 + c] = pool[krow * 8 + c];
+  v_out[orow * 8 + c] = pool[vrow * 8 + c];
+}
+
+cudaError_t launch_append(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                          __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,
+                          int32_t* err, int32_t batch, int32_t max_blocks, int32_t num_pages,
+                          cudaStream_t stream) {
+  if (batch == 0) return cudaSuccess;
+  append_kernel<<<batch, 128, 0, stream>>>(reinterpret_cast<const uint4*>(k_new),
+                                           reinterpret_cast<const uint4*>(v_new),
+                                           reinterpret_cast<uint4*>(pool), bt, seq_lens, err,
+                                           max_blocks, num_pages);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,
+                          __nv_bfloat16* k_out, __nv_bfloat16* v_out, int32_t* err,
+                          int32_t batch, int32_t max_blocks, int32_t num_pages,
+                          int32_t max_seq_len, cudaStream_t stream) {
+  if (batch == 0 || max_seq_len == 0) return cudaSuccess;
+  dim3 grid((max_seq_len + 31) / 32, kKvHeads, batch);
+  gather_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(pool), bt, seq_lens,
+                                          reinterpret_cast<uint4*>(k_out),
+                                          reinterpret_cast<uint4*>(v_out), err, max_blocks,
+                                          num_pages, max_seq_len);
+  return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -1,0 +1,265 @@
+// pkv_api.cu -- the C ABI of pkv.h: argument checks, pool handles, launches.
+//
+// Host-visible argument errors are caught here before anything is launched;
+// everything else is the kernels' business (see pkv.h for the contract).
+#include <new>
+
+#include "pkv_internal.cuh"
+
+struct pkv_pool {
+  void* data;
+  bool owns_data;
+  int32_t num_pages;
+  int device;
+  int sm_count;
+  int32_t* d_err;
+  CUtensorMap tmap;  // 2-D view of the pool: 64 BF16 x (num_pages * 256) rows
+};
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The pool's device must be current for calls that launch on it.
+int check_device(const pkv_pool* pool) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  return dev == pool->device ? PKV_OK : PKV_ERR_INVALID_ARG;
+}
+
+int check_table_args(const pkv_pool* pool, const int32_t* bt, const int32_t* seq_lens,
+                     int32_t layer, int32_t num_layers, int32_t batch, int32_t max_blocks) {
+  if (!pool || !bt || !seq_lens) return PKV_ERR_INVALID_ARG;
+  if (batch < 0 || max_blocks < 1 || num_layers < 1) return PKV_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= num_layers) return PKV_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(batch) * max_blocks * pkv::kKvHeads >= (int64_t(1) << 31))
+    return PKV_ERR_UNSUPPORTED;
+  return check_device(pool);
+}
+
+const int32_t* layer_slab(const int32_t* bt, int32_t layer, int32_t batch, int32_t max_blocks) {
+  return bt + static_cast<int64_t>(layer) * batch * max_blocks;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int pkv_pool_create(int32_t num_pages, int32_t page_tokens, int32_t num_kv_heads,
+                    int32_t head_dim, void* device_storage, size_t storage_bytes,
+                    pkv_pool** out) {
+  if (!out) return PKV_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (page_tokens != PKV_PAGE_TOKENS || num_kv_heads != PKV_NUM_KV_HEADS ||
+      head_dim != PKV_HEAD_DIM)
+    return PKV_ERR_UNSUPPORTED;
+  if (num_pages < 1) return PKV_ERR_INVALID_ARG;
+  // TMA row coordinates (page * 256 + ...) must stay below 2^31.
+  if (static_cast<int64_t>(num_pages) * pkv::kRowsPerPage >= (int64_t(1) << 31))
+    return PKV_ERR_UNSUPPORTED;
+  const size_t need = static_cast<size_t>(num_pages) * PKV_PAGE_BYTES;
+  if (device_storage && (storage_bytes < need || !aligned(device_storage, 16)))
+    return PKV_ERR_INVALID_ARG;
+  EncodeTiledFn encode = encode_tiled_fn();
+  if (!encode) return PKV_ERR_CUDA;
+
+  pkv_pool* p = new (std::nothrow) pkv_pool();
+  if (!p) return PKV_ERR_INVALID_ARG;
+  p->num_pages = num_pages;
+  if (cudaGetDevice(&p->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
+          cudaSuccess) {
+    delete p;
+    return PKV_ERR_CUDA;
+  }
+  if (pkv::prepare_decode_kernels(p->device) != cudaSuccess) {
+    delete p;
+    return PKV_ERR_CUDA;
+  }
+  if (device_storage) {
+    p->data = device_storage;
+    p->owns_data = false;
+  } else {
+    if (cudaMalloc(&p->data, need) != cudaSuccess) {
+      delete p;
+      return PKV_ERR_CUDA;
+    }
+    p->owns_data = true;
+  }
+  if (cudaMalloc(&p->d_err, sizeof(int32_t)) != cudaSuccess ||
+      cudaMemset(p->d_err, 0, sizeof(int32_t)) != cudaSuccess) {
+    if (p->owns_data) cudaFree(p->data);
+    delete p;
+    return PKV_ERR_CUDA;
+  }
+  const cuuint64_t dims[2] = {PKV_HEAD_DIM,
+                              static_cast<cuuint64_t>(num_pages) * pkv::kRowsPerPage};
+  const cuuint64_t strides[1] = {pkv::kRowBytes};
+  const cuuint32_t box[2] = {PKV_HEAD_DIM, PKV_PAGE_TOKENS};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  CUresult r = encode(&p->tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->data, dims, strides, box,
+                      elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    cudaFree(p->d_err);
+    if (p->owns_data) cudaFree(p->data);
+    delete p;
+    return PKV_ERR_CUDA;
+  }
+  *out = p;
+  return PKV_OK;
+}
+
+int pkv_pool_destroy(pkv_pool* pool) {
+  if (!pool) return PKV_OK;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(pool->device);
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaFree(pool->d_err);
+  if (pool->owns_data) cudaFree(pool->data);
+  if (prev >= 0) cudaSetDevice(prev);
+  delete pool;
+  return from_cuda(e);
+}
+
+void* pkv_pool_data(const pkv_pool* pool) { return pool ? pool->data : nullptr; }
+
+int32_t pkv_pool_num_pages(const pkv_pool* pool) { return pool ? pool->num_pages : -1; }
+
+int pkv_append(pkv_pool* pool, const int32_t* block_tables, const int32_t* seq_lens,
+               const uint16_t* k_new, const uint16_t* v_new, int32_t layer, int32_t num_layers,
+               int32_t batch, int32_t max_blocks, pkv_stream_t stream) {
+  int s = check_table_args(pool, block_tables, seq_lens, layer, num_layers, batch, max_blocks);
+  if (s != PKV_OK) return s;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return PKV_ERR_INVALID_ARG;
+  if (batch > 2147483647 / 2) return PKV_ERR_UNSUPPORTED;
+  return from_cuda(pkv::launch_append(
+      reinterpret_cast<const __nv_bfloat16*>(k_new), reinterpret_cast<const __nv_bfloat16*>(v_new),
+      static_cast<__nv_bfloat16*>(pool->data), layer_slab(block_tables, layer, batch, max_blocks),
+      seq_lens, pool->d_err, batch, max_blocks, pool->num_pages,
+      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pkv_decode_workspace_bytes_ex(const pkv_pool* pool, int32_t batch, int32_t kernel,
+                                  int32_t grid_ctas, size_t* bytes_out) {
+  if (!pool || !bytes_out || batch < 0 || grid_ctas < 0) return PKV_ERR_INVALID_ARG;
+  pkv::DecodePlan plan;
+  int s = pkv::plan_decode(pool->device, pool->sm_count, batch, kernel, grid_ctas, &plan);
+  if (s != PKV_OK) return s;
+  *bytes_out = plan.ws_bytes;
+  return PKV_OK;
+}
+
+int pkv_decode_workspace_bytes(const pkv_pool* pool, int32_t batch, size_t* bytes_out) {
+  return pkv_decode_workspace_bytes_ex(pool, batch, PKV_KERNEL_AUTO, 0, bytes_out);
+}
+
+int paged_attention_decode_ex(const uint16_t* q, const pkv_pool* pool,
+                              const int32_t* block_tables, const int32_t* seq_lens, int32_t layer,
+                              float scale, float* out, int32_t num_layers, int32_t batch,
+                              int32_t max_blocks, void* workspace, size_t workspace_bytes,
+                              pkv_stream_t stream, int32_t kernel, int32_t grid_ctas,
+                              int32_t min_chunk) {
+  int s = check_table_args(pool, block_tables, seq_lens, layer, num_layers, batch, max_blocks);
+  if (s != PKV_OK) return s;
+  if (!q || !out || !aligned(q, 16) || !aligned(out, 16)) return PKV_ERR_INVALID_ARG;
+  if (!(scale == scale) || grid_ctas < 0 || min_chunk < 0) return PKV_ERR_INVALID_ARG;
+  if (batch == 0) return PKV_OK;
+  pkv::DecodePlan plan;
+  s = pkv::plan_decode(pool->device, pool->sm_count, batch, kernel, grid_ctas, &plan);
+  if (s != PKV_OK) return s;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < plan.ws_bytes)
+    return PKV_ERR_WORKSPACE;
+  pkv::DecodeArgs a;
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.bt = layer_slab(block_tables, layer, batch, max_blocks);
+  a.seq_lens = seq_lens;
+  a.out = out;
+  a.counters = static_cast<int32_t*>(workspace);
+  a.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.counters_bytes);
+  a.err = pool->d_err;
+  a.batch = batch;
+  a.max_blocks = max_blocks;
+  a.num_pages = pool->num_pages;
+  a.min_chunk = min_chunk;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  return from_cuda(pkv::launch_decode(plan, pool->tmap, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int paged_attention_decode(const uint16_t* q, const pkv_pool* pool, const int32_t* block_tables,
+                           const int32_t* seq_lens, int32_t layer, float scale, float* out,
+                           int32_t num_layers, int32_t batch, int32_t max_blocks,
+                           void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+  return paged_attention_decode_ex(q, pool, block_tables, seq_lens, layer, scale, out, num_layers,
+                                   batch, max_blocks, workspace, workspace_bytes, stream,
+                                   PKV_KERNEL_AUTO, 0, 0);
+}
+
+int pkv_gather(const pkv_pool* pool, const int32_t* block_tables, const int32_t* seq_lens,
+               int32_t layer, uint16_t* k_out, uint16_t* v_out, int32_t num_layers,
+               int32_t batch, int32_t max_blocks, int32_t max_seq_len, pkv_stream_t stream) {
+  int s = check_table_args(pool, block_tables, seq_lens, layer, num_layers, batch, max_blocks);
+  if (s != PKV_OK) return s;
+  if (!k_out || !v_out || !aligned(k_out, 16) || !aligned(v_out, 16) || max_seq_len < 0)
+    return PKV_ERR_INVALID_ARG;
+  if (batch > 65535) return PKV_ERR_UNSUPPORTED;
+  return from_cuda(pkv::launch_gather(
+      static_cast<const __nv_bfloat16*>(pool->data),
+      layer_slab(block_tables, layer, batch, max_blocks), seq_lens,
+      reinterpret_cast<__nv_bfloat16*>(k_out), reinterpret_cast<__nv_bfloat16*>(v_out),
+      pool->d_err, batch, max_blocks, pool->num_pages, max_seq_len,
+      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pkv_get_device_error(pkv_pool* pool, pkv_stream_t stream, int32_t* status_out) {
+  if (!pool || !status_out) return PKV_ERR_INVALID_ARG;
+  int s = check_device(pool);
+  if (s != PKV_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&v, pool->d_err, sizeof v, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(pool->d_err, 0, sizeof(int32_t), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return PKV_ERR_CUDA;
+  *status_out = v;
+  return PKV_OK;
+}
+
+const char* pkv_status_string(int status) {
+  switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_INVALID_ARG: return "invalid argument";
+    case PKV_ERR_UNSUPPORTED: return "unsupported shape or size";
+    case PKV_ERR_CUDA: return "CUDA runtime error";
+    case PKV_ERR_OUT_OF_PAGES: return "out of pages";
+    case PKV_ERR_BAD_PAGE: return "block-table entry outside the pool";
+    case PKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case PKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case PKV_ERR_BAD_SEQ_LEN: return "sequence length out of range";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,174 @@
+// pkv_internal.cuh -- shared definitions of the sm_100a kernels behind pkv.h.
+//
+// Shapes: 16-token pages ("Curso gratuito recorre la inferencia de LLM...",
+// section on the KV cache), 32 query heads over 8 kv heads of dimension 64
+// ("Construye tu propio motor de inferencia LLM...", sections on the
+// Llama 3.2 1B architecture and on GQA).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pkv.h"
+
+namespace pkv {
+
+constexpr int kTokens = 16;                       // tokens per page
+constexpr int kKvHeads = 8;
+constexpr int kQHeads = 32;
+constexpr int kDim = 64;
+constexpr int kGroup = kQHeads / kKvHeads;        // 4 query heads per kv head
+constexpr int kRowBytes = kDim * 2;               // one token of one kv head: 128 B
+constexpr int kTileBytes = kTokens * kRowBytes;   // (page, K|V, kv head) tile: 2 KiB
+constexpr int kRowsPerPage = 2 * kKvHeads * kTokens;  // 256 rows of 128 B
+constexpr int kPartialFloats = 2 * kGroup + kGroup * kDim;  // m[4], l[4], acc[4][64]
+
+// Sticky device error codes (first one wins).
+constexpr int32_t kErrBadPage = PKV_ERR_BAD_PAGE;
+constexpr int32_t kErrBadLen = PKV_ERR_BAD_SEQ_LEN;
+constexpr int32_t kErrTimeout = PKV_ERR_DEVICE_TIMEOUT;
+
+// Bounded waits give up after this many nanoseconds of global time.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+__device__ __forceinline__ void record_error(int32_t* err, int32_t code) {
+  atomicCAS(err, 0, code);
+}
+
+// ------------------------------------------------------------ PTX wrappers --
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of an mbarrier; false once kWaitLimitNs have
+// passed without completion (the caller records kErrTimeout).
+static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// L2 policy for data read exactly once (the KV stream).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 2-D tiled TMA load (no multicast) of box {64 elements, 16 rows} at
+// coordinates (x, y) into shared memory, completing on mbarrier `bar`.
+__device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* map, int32_t x,
+                                              int32_t y, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// Byte offset of 16-byte chunk `c` of row `r` inside a TMA tile written with
+// the 128-byte swizzle (rows of 128 B; chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return static_cast<uint32_t>(r * kRowBytes + ((c ^ (r & 7)) << 4));
+}
+
+// BF16 pair (one 32-bit word, element 0 in the low half) -> two floats.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// ------------------------------------------------------------ launch glue --
+
+struct DecodeArgs {
+  const __nv_bfloat16* q;   // [B][32][64]
+  const int32_t* bt;        // this layer's block-table slab [B][max_blocks]
+  const int32_t* seq_lens;  // [B]
+  float* out;               // [B][32][64]
+  float* partials;          // [8B + W - 1][kPartialFloats]
+  int32_t* counters;        // [8B]
+  int32_t* err;             // sticky device error word
+  int32_t batch;
+  int32_t max_blocks;
+  int32_t num_pages;
+  int32_t min_chunk;        // minimum (page, kv head) tiles per warp
+  float scale_log2;         // scale * log2(e)
+};
+
+// Launch planning shared by the workspace query and the launch.
+struct DecodePlan {
+  int kernel;        // PKV_KERNEL_SIMT or PKV_KERNEL_MMA
+  int grid;          // CTAs
+  int warps;         // warps per CTA
+  size_t smem;       // dynamic shared memory bytes
+  size_t ws_bytes;   // workspace bytes
+  size_t counters_bytes;
+};
+
+int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,
+                DecodePlan* plan);
+cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const DecodeArgs& a,
+                          cudaStream_t stream);
+cudaError_t prepare_decode_kernels(int device);
+
+cudaError_t launch_append(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                          __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,
+                          int32_t* err, int32_t batch, int32_t max_blocks, int32_t num_pages,
+                          cudaStream_t stream);
+
+cudaError_t launch_gather(const __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,
+                          __nv_bfloat16* k_out, __nv_bfloat16* v_out, int32_t* err,
+                          int32_t batch, int32_t max_blocks, int32_t num_pages,
+                          int32_t max_seq_len, cudaStream_t stream);
+
+}  // namespace pkv

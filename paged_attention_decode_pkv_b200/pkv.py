@@ -1,0 +1,224 @@
+"""Python binding of libpkv (the C ABI in include/pkv.h).
+
+Argument marshalling only: every step of append, gather and decode runs in
+the CUDA kernels of libpkv.so.  Tensors are torch CUDA tensors; torch is used
+for device memory and streams, nothing else.  There is no CPU fallback: if
+libpkv.so is missing or cannot be loaded, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkv.so")
+
+PAGE_TOKENS = 16
+NUM_KV_HEADS = 8
+NUM_Q_HEADS = 32
+HEAD_DIM = 64
+PAGE_BYTES = 32768
+
+KERNEL_AUTO, KERNEL_SIMT, KERNEL_MMA = 0, 1, 2
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_CUDA = -3
+ERR_OUT_OF_PAGES = -4
+ERR_BAD_PAGE = -5
+ERR_WORKSPACE = -6
+ERR_DEVICE_TIMEOUT = -7
+ERR_BAD_SEQ_LEN = -8
+
+EXPORTS = (
+    "pkv_pool_create", "pkv_pool_destroy", "pkv_pool_data", "pkv_pool_num_pages", "pkv_append",
+    "pkv_decode_workspace_bytes", "pkv_decode_workspace_bytes_ex", "paged_attention_decode",
+    "paged_attention_decode_ex", "pkv_gather", "pkv_get_device_error", "pkv_status_string",
+)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libpkv.so not built at %s (run python -m "
+                          "paged_attention_decode_pkv_b200.build)" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    sig = {
+        "pkv_pool_create": ([i32, i32, i32, i32, P, sz, ctypes.POINTER(P)], ctypes.c_int),
+        "pkv_pool_destroy": ([P], ctypes.c_int),
+        "pkv_pool_data": ([P], P),
+        "pkv_pool_num_pages": ([P], i32),
+        "pkv_append": ([P, P, P, P, P, i32, i32, i32, i32, P], ctypes.c_int),
+        "pkv_decode_workspace_bytes": ([P, i32, ctypes.POINTER(sz)], ctypes.c_int),
+        "pkv_decode_workspace_bytes_ex": ([P, i32, i32, i32, ctypes.POINTER(sz)], ctypes.c_int),
+        "paged_attention_decode": ([P, P, P, P, i32, ctypes.c_float, P, i32, i32, i32, P, sz, P],
+                                   ctypes.c_int),
+        "paged_attention_decode_ex": ([P, P, P, P, i32, ctypes.c_float, P, i32, i32, i32, P, sz,
+                                       P, i32, i32, i32], ctypes.c_int),
+        "pkv_gather": ([P, P, P, i32, P, P, i32, i32, i32, i32, P], ctypes.c_int),
+        "pkv_get_device_error": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
+        "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+lib = _load()
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        msg = lib.pkv_status_string(status).decode()
+        super().__init__("%s%s (status %d)" % (what + ": " if what else "", msg, status))
+        self.status = status
+
+
+def status_string(status: int) -> str:
+    return lib.pkv_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise PkvError(status, what)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, shape, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Pool:
+    """A pool of 32 KiB pages ([K|V][8 kv heads][16 slots][64] BF16 each).
+
+    The page storage is a torch tensor owned by this object
+    (``self.storage``, bfloat16 [num_pages, 2, 8, 16, 64]) or one the caller
+    passes in; the C library only borrows it.
+    """
+
+    def __init__(self, num_pages: int, storage: Optional[torch.Tensor] = None, device=None):
+        if storage is None:
+            storage = torch.empty((num_pages, 2, NUM_KV_HEADS, PAGE_TOKENS, HEAD_DIM),
+                                  dtype=torch.bfloat16, device=device or "cuda")
+        _dev(storage, torch.bfloat16, (num_pages, 2, NUM_KV_HEADS, PAGE_TOKENS, HEAD_DIM),
+             "storage")
+        self.storage = storage
+        self.num_pages = int(num_pages)
+        self.device = storage.device
+        self._h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            _check(lib.pkv_pool_create(num_pages, PAGE_TOKENS, NUM_KV_HEADS, HEAD_DIM,
+                                       ctypes.c_void_p(storage.data_ptr()),
+                                       storage.numel() * 2, ctypes.byref(self._h)),
+                   "pkv_pool_create")
+        self._ws = {}
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if not self._h:
+            raise RuntimeError("pool destroyed")
+        return self._h
+
+    def close(self):
+        if self._h:
+            with torch.cuda.device(self.device):
+                lib.pkv_pool_destroy(self._h)
+            self._h = ctypes.c_void_p()
+        self._ws.clear()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self, batch: int, kernel: int = KERNEL_AUTO, grid_ctas: int = 0) -> int:
+        n = ctypes.c_size_t()
+        with torch.cuda.device(self.device):
+            _check(lib.pkv_decode_workspace_bytes_ex(self.handle, int(batch), int(kernel),
+                                                     int(grid_ctas), ctypes.byref(n)),
+                   "pkv_decode_workspace_bytes")
+        return n.value
+
+    def workspace(self, batch: int, kernel: int = KERNEL_AUTO, grid_ctas: int = 0) -> torch.Tensor:
+        """A zero-initialised workspace, cached per (batch, kernel, grid)."""
+        key = (int(batch), int(kernel), int(grid_ctas))
+        ws = self._ws.get(key)
+        if ws is None:
+            ws = torch.zeros(max(256, self.workspace_bytes(*key)), dtype=torch.uint8,
+                             device=self.device)
+            self._ws[key] = ws
+        return ws
+
+
+def append(pool: Pool, block_tables: torch.Tensor, seq_lens: torch.Tensor, k_new: torch.Tensor,
+           v_new: torch.Tensor, layer: int, stream=None):
+    L, B, MB = block_tables.shape
+    _check(lib.pkv_append(pool.handle, _dev(block_tables, torch.int32, None, "block_tables"),
+                          _dev(seq_lens, torch.int32, (B,), "seq_lens"),
+                          _dev(k_new, torch.bfloat16, (B, NUM_KV_HEADS, HEAD_DIM), "k_new"),
+                          _dev(v_new, torch.bfloat16, (B, NUM_KV_HEADS, HEAD_DIM), "v_new"),
+                          int(layer), L, B, MB, _stream(stream)), "pkv_append")
+
+
+def decode(q: torch.Tensor, pool: Pool, block_tables: torch.Tensor, seq_lens: torch.Tensor,
+           layer: int, scale: float, out: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None, kernel: int = KERNEL_AUTO,
+           grid_ctas: int = 0, min_chunk: int = 0, stream=None) -> torch.Tensor:
+    L, B, MB = block_tables.shape
+    if out is None:
+        out = torch.empty((B, NUM_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = pool.workspace(B, kernel, grid_ctas)
+    _check(lib.paged_attention_decode_ex(
+        _dev(q, torch.bfloat16, (B, NUM_Q_HEADS, HEAD_DIM), "q"), pool.handle,
+        _dev(block_tables, torch.int32, None, "block_tables"),
+        _dev(seq_lens, torch.int32, (B,), "seq_lens"), int(layer), float(scale),
+        _dev(out, torch.float32, (B, NUM_Q_HEADS, HEAD_DIM), "out"), L, B, MB,
+        _dev(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream),
+        int(kernel), int(grid_ctas), int(min_chunk)), "paged_attention_decode")
+    return out
+
+
+def gather(pool: Pool, block_tables: torch.Tensor, seq_lens: torch.Tensor, layer: int,
+           max_seq_len: int, k_out: Optional[torch.Tensor] = None,
+           v_out: Optional[torch.Tensor] = None, stream=None):
+    L, B, MB = block_tables.shape
+    shape = (B, NUM_KV_HEADS, max_seq_len, HEAD_DIM)
+    if k_out is None:
+        k_out = torch.zeros(shape, dtype=torch.bfloat16, device=pool.device)
+    if v_out is None:
+        v_out = torch.zeros(shape, dtype=torch.bfloat16, device=pool.device)
+    _check(lib.pkv_gather(pool.handle, _dev(block_tables, torch.int32, None, "block_tables"),
+                          _dev(seq_lens, torch.int32, (B,), "seq_lens"), int(layer),
+                          _dev(k_out, torch.bfloat16, shape, "k_out"),
+                          _dev(v_out, torch.bfloat16, shape, "v_out"), L, B, MB,
+                          int(max_seq_len), _stream(stream)), "pkv_gather")
+    return k_out, v_out
+
+
+def get_device_error(pool: Pool, stream=None) -> int:
+    """Synchronise the stream; return and clear the pool's sticky device error."""
+    v = ctypes.c_int32()
+    _check(lib.pkv_get_device_error(pool.handle, _stream(stream), ctypes.byref(v)),
+           "pkv_get_device_error")
+    return v.value

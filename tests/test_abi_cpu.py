@@ -1,0 +1,67 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol
+include/pkv.h declares, and rejects bad host arguments before touching the
+GPU.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"PKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", src))
+    return names
+
+
+def test_header_declares_the_documented_calls():
+    names = _declared()
+    for n in ("pkv_pool_create", "pkv_append", "paged_attention_decode", "pkv_gather",
+              "pkv_get_device_error", "pkv_decode_workspace_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from paged_attention_decode_pkv_b200 import pkv
+    lib = ctypes.CDLL(pkv.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert set(pkv.EXPORTS) >= _declared()
+
+
+def test_status_strings():
+    from paged_attention_decode_pkv_b200 import pkv
+    assert pkv.status_string(0) == "ok"
+    assert "outside the pool" in pkv.status_string(pkv.ERR_BAD_PAGE)
+    assert pkv.status_string(12345) == "unknown status"
+
+
+def test_pool_create_rejects_bad_shapes_and_null_out():
+    from paged_attention_decode_pkv_b200 import pkv
+    h = ctypes.c_void_p()
+    assert pkv.lib.pkv_pool_create(16, 32, 8, 64, None, 0, ctypes.byref(h)) == pkv.ERR_UNSUPPORTED
+    assert pkv.lib.pkv_pool_create(16, 16, 4, 64, None, 0, ctypes.byref(h)) == pkv.ERR_UNSUPPORTED
+    assert pkv.lib.pkv_pool_create(16, 16, 8, 128, None, 0, ctypes.byref(h)) == pkv.ERR_UNSUPPORTED
+    assert pkv.lib.pkv_pool_create(0, 16, 8, 64, None, 0, ctypes.byref(h)) == pkv.ERR_INVALID_ARG
+    assert pkv.lib.pkv_pool_create(16, 16, 8, 64, None, 0, None) == pkv.ERR_INVALID_ARG
+    # a pool whose TMA row coordinates would overflow int32
+    assert pkv.lib.pkv_pool_create(1 << 23, 16, 8, 64, None, 0, ctypes.byref(h)) == \
+        pkv.ERR_UNSUPPORTED
+
+
+def test_calls_reject_null_pool():
+    from paged_attention_decode_pkv_b200 import pkv
+    P = ctypes.c_void_p(16)
+    assert pkv.lib.pkv_append(None, P, P, P, P, 0, 1, 1, 1, None) == pkv.ERR_INVALID_ARG
+    assert pkv.lib.paged_attention_decode(P, None, P, P, 0, 0.125, P, 1, 1, 1, P, 1 << 20,
+                                          None) == pkv.ERR_INVALID_ARG
+    assert pkv.lib.pkv_gather(None, P, P, 0, P, P, 1, 1, 1, 16, None) == pkv.ERR_INVALID_ARG
+    n = ctypes.c_size_t()
+    assert pkv.lib.pkv_decode_workspace_bytes(None, 4, ctypes.byref(n)) == pkv.ERR_INVALID_ARG
+    assert pkv.lib.pkv_pool_destroy(None) == pkv.OK
+    assert pkv.lib.pkv_pool_num_pages(None) == -1

@@ -1,0 +1,161 @@
+"""GPU parity on small cases: CUDA path (through the C ABI) vs the FP64
+oracle, on the same BF16 input bits.  Covers ragged lengths around page
+boundaries, empty sequences, forced split-KV patterns, NaN in every slot
+outside the context, bit-exact append and gather, device-side error reports
+and launch-to-launch determinism."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_attention_decode_pkv_b200 import pkv
+from paged_attention_decode_pkv_b200 import workloads as W
+from tests.cases import NAN, bf16_bits, make_case
+from tests.harness import ATOL, KERNELS, GpuCase, bits, max_err, to_dev, u16_to_bf16
+
+pytestmark = pytest.mark.gpu
+
+EDGE_LENS = [[1], [15], [16], [17], [31], [32], [33], [0, 5], [1, 15, 16, 17, 31, 32, 33, 0, 64],
+             [200, 3, 77, 1000, 16]]
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("lens", EDGE_LENS)
+def test_decode_edge_lengths(kernel, lens):
+    g = GpuCase(make_case(lens, seed=len(lens) * 100 + sum(lens), spare_pages=5))
+    got = g.decode(kernel=kernel)
+    want = g.oracle()
+    assert np.isfinite(got).all()
+    assert max_err(got, want) <= ATOL
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert not got[b].any()
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("grid,min_chunk", [(1, 0), (2, 0), (7, 0), (3, 1), (0, 1), (0, 3),
+                                            (0, 64), (50, 2)])
+def test_decode_split_patterns(kernel, grid, min_chunk):
+    # Different grids / chunk sizes cut the (sequence, kv head) runs at
+    # different places, exercising the split-KV merge; the result must stay
+    # within tolerance of the oracle for every cut.
+    g = GpuCase(make_case([300, 1, 47, 129, 16, 517], seed=77, spare_pages=9))
+    want = g.oracle(scale=0.09)
+    got = g.decode(scale=0.09, kernel=kernel, grid_ctas=grid, min_chunk=min_chunk)
+    assert max_err(got, want) <= ATOL
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_tiny_workload_append_and_decode(kernel):
+    w = W.tiny()
+    dev = "cuda"
+    pool_t = W.make_pool(w, dev)
+    host_pool = bits(pool_t).reshape(w.num_pages, 2, 8, 16, 64).copy()
+    pool = pkv.Pool(w.num_pages, storage=pool_t)
+    bt = to_dev(w.block_tables)
+    sl_np = w.seq_lens(1)
+    sl = to_dev(sl_np)
+    q, k, v = W.step_inputs(w, 1, 0, dev)
+    pkv.append(pool, bt, sl, k, v, 0)
+    out = pkv.decode(q, pool, bt, sl, 0, w.scale, kernel=kernel)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error(pool) == 0
+    oracle.append(host_pool, w.block_tables, sl_np, bits(k), bits(v), 0)
+    assert np.array_equal(bits(pool_t).reshape(host_pool.shape), host_pool)   # whole pool
+    want = oracle.decode(bits(q), host_pool, w.block_tables, sl_np, 0, w.scale)
+    assert max_err(out.cpu().numpy().astype(np.float64), want) <= ATOL
+
+
+def test_append_bit_exact_and_touches_nothing_else():
+    c = make_case([17, 40, 1, 16, 33], seed=5, spare_pages=7, num_layers=2)
+    g = GpuCase(c)
+    rng = np.random.default_rng(0)
+    k = bf16_bits(rng.standard_normal((5, 8, 64)))
+    v = bf16_bits(rng.standard_normal((5, 8, 64)))
+    host = c["pool"].copy()
+    for layer in (1, 0):
+        pkv.append(g.pool, g.bt, g.sl, u16_to_bf16(k), u16_to_bf16(v), layer)
+        oracle.append(host, c["bt"], c["seq_lens"], k, v, layer)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error(g.pool) == 0
+    assert np.array_equal(bits(g.pool_t).reshape(host.shape), host)
+
+
+def test_gather_bit_exact_and_leaves_tail():
+    c = make_case([17, 40, 0, 33, 1], seed=9, spare_pages=4, num_layers=3)
+    g = GpuCase(c)
+    for layer in range(3):
+        k0 = np.full((5, 8, 48, 64), 0x1234, np.uint16)
+        v0 = np.full((5, 8, 48, 64), 0x4321, np.uint16)
+        kd, vd = u16_to_bf16(k0), u16_to_bf16(v0)
+        pkv.gather(g.pool, g.bt, g.sl, layer, 48, kd, vd)
+        ko, vo = oracle.gather(c["pool"], c["bt"], c["seq_lens"], layer, 48, k0.copy(), v0.copy())
+        assert np.array_equal(bits(kd).reshape(ko.shape), ko)
+        assert np.array_equal(bits(vd).reshape(vo.shape), vo)
+    assert pkv.get_device_error(g.pool) == 0
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_nan_outside_context_never_reaches_output(kernel):
+    c = make_case([1, 15, 17, 31, 49], seed=11, spare_pages=8)
+    assert (c["pool"] == NAN).sum() > 0
+    g = GpuCase(c)
+    got = g.decode(kernel=kernel)
+    assert np.isfinite(got).all()
+    assert max_err(got, g.oracle()) <= ATOL
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_repeated_launches_are_bitwise_identical(kernel):
+    g = GpuCase(make_case([700, 33, 1, 260, 95, 16, 17], seed=13, spare_pages=3))
+    ref = g.decode(kernel=kernel, grid_ctas=5)
+    for _ in range(100):
+        assert np.array_equal(g.decode(kernel=kernel, grid_ctas=5), ref)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_bad_page_is_reported_not_faulted(kernel):
+    c = make_case([40, 20], seed=17, spare_pages=2)
+    bad = c["bt"].copy()
+    bad[0, 0, 1] = 1 << 20          # far outside the pool
+    g = GpuCase(dict(c, bt=bad))
+    got = g.decode(kernel=kernel)
+    assert pkv.get_device_error(g.pool) == pkv.ERR_BAD_PAGE
+    # the other sequence is unaffected
+    want = oracle.decode(c["q"], c["pool"], c["bt"], c["seq_lens"], 0, 0.125)
+    assert max_err(got[1], want[1]) <= ATOL
+    pkv.append(g.pool, g.bt, g.sl, u16_to_bf16(c["k_new"]), u16_to_bf16(c["v_new"]), 0)
+    assert pkv.get_device_error(g.pool) in (pkv.ERR_BAD_PAGE, 0)
+    assert pkv.get_device_error(g.pool) == 0       # cleared by the previous read
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_bad_seq_len_is_reported_and_row_zeroed(kernel):
+    c = make_case([40, 20], seed=19, spare_pages=2)
+    g = GpuCase(c)
+    g.sl = to_dev(np.array([40, 10_000], np.int32))
+    got = g.decode(kernel=kernel)
+    assert pkv.get_device_error(g.pool) == pkv.ERR_BAD_SEQ_LEN
+    assert not got[1].any()
+    assert max_err(got[0], g.oracle()[0]) <= ATOL
+    g.sl = to_dev(np.array([0, 20], np.int32))
+    pkv.append(g.pool, g.bt, g.sl, u16_to_bf16(c["k_new"]), u16_to_bf16(c["v_new"]), 0)
+    assert pkv.get_device_error(g.pool) == pkv.ERR_BAD_SEQ_LEN
+
+
+def test_workspace_too_small_is_rejected():
+    g = GpuCase(make_case([40, 20], seed=23))
+    need = g.pool.workspace_bytes(2)
+    ws = torch.zeros(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pkv.PkvError) as e:
+        pkv.decode(g.q, g.pool, g.bt, g.sl, 0, 0.125, workspace=ws)
+    assert e.value.status == pkv.ERR_WORKSPACE
+
+
+def test_scale_and_layer_arguments():
+    c = make_case([33, 70], seed=29, num_layers=3, spare_pages=2)
+    g = GpuCase(c)
+    for layer in range(3):
+        for scale in (0.0, 0.125, 0.5):
+            got = g.decode(layer=layer, scale=scale)
+            assert max_err(got, g.oracle(layer=layer, scale=scale)) <= ATOL
