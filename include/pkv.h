@@ -197,6 +197,10 @@ PKV_API int pkv_get_device_error(pkv_pool *pool, pkv_stream_t stream, int32_t *s
 /* Static English text for a status code. */
 PKV_API const char *pkv_status_string(int status);
 
+/* Text naming the CUDA call behind the calling thread's most recent
+ * PKV_ERR_CUDA ("" if none); valid until the thread's next failing call. */
+PKV_API const char *pkv_last_error_message(void);
+
 #ifdef __cplusplus
 }
 #endif

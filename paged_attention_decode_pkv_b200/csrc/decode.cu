@@ -551,7 +551,11 @@ cudaError_t prepare_decode_kernels(int device) {
   cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
   if (e != cudaSuccess) return e;
   for (int k : {PKV_KERNEL_SIMT}) {
-    e = cudaFuncSetAttribute(kernel_for(k), cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kernel_for(k));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel_for(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - static_cast<int>(fa.sharedSizeBytes));
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -567,7 +571,9 @@ int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ct
       cudaSuccess)
     return PKV_ERR_CUDA;
   const size_t smem = decode_smem_bytes(batch);
-  if (smem > static_cast<size_t>(optin)) return PKV_ERR_UNSUPPORTED;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return PKV_ERR_CUDA;
+  if (smem + fa.sharedSizeBytes > static_cast<size_t>(optin)) return PKV_ERR_UNSUPPORTED;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kWarps * 32, smem) !=
       cudaSuccess)

@@ -2,6 +2,7 @@
 //
 // Host-visible argument errors are caught here before anything is launched;
 // everything else is the kernels' business (see pkv.h for the contract).
+#include <cstdio>
 #include <new>
 
 #include "pkv_internal.cuh"
@@ -59,7 +60,17 @@ const int32_t* layer_slab(const int32_t* bt, int32_t layer, int32_t batch, int32
   return bt + static_cast<int64_t>(layer) * batch * max_blocks;
 }
 
-int from_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
+thread_local char g_last_error[256] = "";
+
+void note(const char* where, cudaError_t e) {
+  snprintf(g_last_error, sizeof g_last_error, "%s: %s", where, cudaGetErrorString(e));
+}
+
+int from_cuda(cudaError_t e, const char* where = "kernel launch") {
+  if (e == cudaSuccess) return PKV_OK;
+  note(where, e);
+  return PKV_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -81,36 +92,43 @@ int pkv_pool_create(int32_t num_pages, int32_t page_tokens, int32_t num_kv_heads
   if (device_storage && (storage_bytes < need || !aligned(device_storage, 16)))
     return PKV_ERR_INVALID_ARG;
   EncodeTiledFn encode = encode_tiled_fn();
-  if (!encode) return PKV_ERR_CUDA;
+  if (!encode) {
+    snprintf(g_last_error, sizeof g_last_error, "pkv_pool_create: cuTensorMapEncodeTiled not found");
+    return PKV_ERR_CUDA;
+  }
 
   pkv_pool* p = new (std::nothrow) pkv_pool();
   if (!p) return PKV_ERR_INVALID_ARG;
   p->num_pages = num_pages;
-  if (cudaGetDevice(&p->device) != cudaSuccess ||
-      cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device) !=
-          cudaSuccess) {
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device);
+  if (e != cudaSuccess) {
     delete p;
-    return PKV_ERR_CUDA;
+    return from_cuda(e, "pkv_pool_create: device query");
   }
-  if (pkv::prepare_decode_kernels(p->device) != cudaSuccess) {
+  e = pkv::prepare_decode_kernels(p->device);
+  if (e != cudaSuccess) {
     delete p;
-    return PKV_ERR_CUDA;
+    return from_cuda(e, "pkv_pool_create: kernel attributes");
   }
   if (device_storage) {
     p->data = device_storage;
     p->owns_data = false;
   } else {
-    if (cudaMalloc(&p->data, need) != cudaSuccess) {
+    e = cudaMalloc(&p->data, need);
+    if (e != cudaSuccess) {
       delete p;
-      return PKV_ERR_CUDA;
+      return from_cuda(e, "pkv_pool_create: cudaMalloc(pool)");
     }
     p->owns_data = true;
   }
-  if (cudaMalloc(&p->d_err, sizeof(int32_t)) != cudaSuccess ||
-      cudaMemset(p->d_err, 0, sizeof(int32_t)) != cudaSuccess) {
+  e = cudaMalloc(&p->d_err, sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaMemset(p->d_err, 0, sizeof(int32_t));
+  if (e != cudaSuccess) {
     if (p->owns_data) cudaFree(p->data);
     delete p;
-    return PKV_ERR_CUDA;
+    return from_cuda(e, "pkv_pool_create: error word");
   }
   const cuuint64_t dims[2] = {PKV_HEAD_DIM,
                               static_cast<cuuint64_t>(num_pages) * pkv::kRowsPerPage};
@@ -121,6 +139,8 @@ int pkv_pool_create(int32_t num_pages, int32_t page_tokens, int32_t num_kv_heads
                       elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof g_last_error, "pkv_pool_create: cuTensorMapEncodeTiled: CUresult %d",
+             static_cast<int>(r));
     cudaFree(p->d_err);
     if (p->owns_data) cudaFree(p->data);
     delete p;
@@ -246,6 +266,8 @@ int pkv_get_device_error(pkv_pool* pool, pkv_stream_t stream, int32_t* status_ou
   *status_out = v;
   return PKV_OK;
 }
+
+const char* pkv_last_error_message(void) { return g_last_error; }
 
 const char* pkv_status_string(int status) {
   switch (status) {

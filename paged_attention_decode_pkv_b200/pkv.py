@@ -38,6 +38,7 @@ EXPORTS = (
     "pkv_pool_create", "pkv_pool_destroy", "pkv_pool_data", "pkv_pool_num_pages", "pkv_append",
     "pkv_decode_workspace_bytes", "pkv_decode_workspace_bytes_ex", "paged_attention_decode",
     "paged_attention_decode_ex", "pkv_gather", "pkv_get_device_error", "pkv_status_string",
+    "pkv_last_error_message",
 )
 
 
@@ -62,6 +63,7 @@ def _load():
         "pkv_gather": ([P, P, P, i32, P, P, i32, i32, i32, i32, P], ctypes.c_int),
         "pkv_get_device_error": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
         "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "pkv_last_error_message": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -76,6 +78,8 @@ lib = _load()
 class PkvError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         msg = lib.pkv_status_string(status).decode()
+        if status == ERR_CUDA:
+            msg += " [%s]" % lib.pkv_last_error_message().decode()
         super().__init__("%s%s (status %d)" % (what + ": " if what else "", msg, status))
         self.status = status
 
