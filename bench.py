@@ -140,28 +140,46 @@ class Runner:
         self.v = torch.stack([x[2] for x in ins])
         self.out = torch.empty((nl, B, 32, 64), dtype=torch.float32, device=device)
         self.ws = self.pool.workspace(B, kernel)
-        self.step_idx = 0
 
-    def step(self, stream, ev_pairs=None):
-        """One decode step over all layers; optionally records (start, end)
-        events around every decode launch."""
+    def launch_step(self, stream, variant, events=None, seq_lens=None):
+        """Launch one decode step (all layers) for lengths variant `variant`;
+        optionally record (start, end) events around every decode launch."""
         pkv = self.pkv
-        sl = self.seq_lens[self.step_idx % self.w.num_steps]
-        self.step_idx += 1
+        sl = self.seq_lens[variant] if seq_lens is None else seq_lens
         for l in range(self.w.num_layers):
             pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
-            if ev_pairs is not None:
-                e0, e1 = ev_pairs.pop()
-                e0.record(stream)
+            if events is not None:
+                events[l][0].record(stream)
             pkv.decode(self.q[l], self.pool, self.bt, sl, l, self.w.scale, out=self.out[l],
                        workspace=self.ws, kernel=self.kernel, stream=stream)
-            if ev_pairs is not None:
-                e1.record(stream)
-                self.used.append((e0, e1))
+            if events is not None:
+                events[l][1].record(stream)
 
-    def step_bytes(self, step_idx):
-        sl = self.w.seq_lens(step_idx % self.w.num_steps + 1)
-        return alg_bytes_decode(sl)
+    def capture(self, stream):
+        """One CUDA graph per lengths variant (the workload's step cycle),
+        each with timing events around its decode launches."""
+        self.graphs, self.events = [], []
+        for v in range(self.w.num_steps):
+            ev = [(torch.cuda.Event(enable_timing=True, external=True),
+                   torch.cuda.Event(enable_timing=True, external=True))
+                  for _ in range(self.w.num_layers)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                self.launch_step(stream, v, ev)
+            self.graphs.append(g)
+            self.events.append(ev)
+
+    def replay(self, i):
+        self.graphs[i % len(self.graphs)].replay()
+
+    def decode_times(self):
+        """(ms, algorithmic bytes) of every decode launch in the last replay
+        of each graph."""
+        out = []
+        for v, ev in enumerate(self.events):
+            nbytes = alg_bytes_decode(self.w.seq_lens(v + 1))
+            out += [(a.elapsed_time(b), nbytes) for a, b in ev]
+        return out
 
 
 def run_ours(args, rank, world, local_rank):
@@ -172,6 +190,9 @@ def run_ours(args, rank, world, local_rank):
     w = W.make(args.workload, seed=W.make(args.workload).seed + 1000 * rank) if rank else \
         W.make(args.workload)
     r = Runner(w, device, kernel)
+    if not args.no_pdl:
+        # appends precede every decode and only read the tables
+        r.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES)
     stream = torch.cuda.Stream(device)
     dist = world > 1
     if dist:
@@ -182,31 +203,32 @@ def run_ours(args, rank, world, local_rank):
             tdist.barrier()
 
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            r.step(stream)
+        for i in range(args.warmup):
+            r.launch_step(stream, i % w.num_steps)
     stream.synchronize()
     assert pkv.get_device_error(r.pool, stream) == 0
+    r.capture(stream)
+    for i in range(max(args.warmup, w.num_steps)):
+        r.replay(i)
+    torch.cuda.synchronize()
 
-    # ---- timed region: K steps, decode launches bracketed by events
-    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps * w.num_layers)]
-    r.used = []
+    # ---- timed region: K graph launches, one decode step each
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    first_step = r.step_idx
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         with torch.cuda.stream(stream):
             t0.record(stream)
-            for _ in range(args.steps):
-                r.step(stream, pairs)
+            for i in range(args.steps):
+                r.replay(i)
             t1.record(stream)
         stream.synchronize()
         torch.cuda.synchronize()
     barrier()
     ms = t0.elapsed_time(t1)
-    dec_ms = [a.elapsed_time(b) for a, b in r.used]
-    dec_bytes = [r.step_bytes(first_step + i // w.num_layers) for i in range(len(dec_ms))]
+    times = r.decode_times()
+    dec_ms = [t for t, _ in times]
+    dec_bytes = [nb for _, nb in times]
     err = pkv.get_device_error(r.pool, stream)
     if err != 0:
         raise RuntimeError("device error during timed region: %s" % pkv.status_string(err))
@@ -235,6 +257,9 @@ def run_ours(args, rank, world, local_rank):
             "layers": w.num_layers, "pool_pages": w.num_pages,
             "kv_bytes_per_layer": w.kv_bytes(1), "accumulate": "f32",
             "kernel": args.kernel, "parallelism": "dp%d (independent replicas)" % world,
+            "launch": "one CUDA graph per step (16 x append + decode + split merge)%s" %
+                      ("" if args.no_pdl else ", programmatic dependent launch, "
+                                             "tables read before the append ends"),
             "l2": "inputs larger than L2: one step reads %.0f MB of K/V" %
                   (w.kv_bytes(1) * w.num_layers / 1e6),
         },
@@ -246,7 +271,9 @@ def run_ours(args, rank, world, local_rank):
         },
         "decode_only_queries_per_s": w.batch / avg_dec_s,
         "e2e": e2e,
-        "gpu_launches": args.steps * w.num_layers * 2,
+        "gpu_launches": args.steps * w.num_layers * 3,
+        "decode_timing": "CUDA events recorded inside the step graphs, last replay of each "
+                         "of the %d graphs (%d decode launches)" % (w.num_steps, len(dec_ms)),
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline:
@@ -255,32 +282,29 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_e2e(r: Runner, stream, steps, barrier, dist, device):
-    """Same step, with every step's inputs (q, k_new, v_new of all layers,
-    seq_lens) copied from pinned host memory and all outputs copied back."""
+    """Same step through the public API, with every step's inputs (q, k_new,
+    v_new of all layers, seq_lens) copied from pinned host memory before the
+    step's graph runs and all outputs copied back to pinned host memory."""
     w = r.w
     hq = r.q.cpu().pin_memory()
     hk = r.k.cpu().pin_memory()
     hv = r.v.cpu().pin_memory()
     hsl = [x.cpu().pin_memory() for x in r.seq_lens]
     hout = torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory()
-    sl_dev = torch.empty_like(r.seq_lens[0])
     h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + hsl[0].numel() * 4
     d2h = hout.numel() * 4
-    pkv = r.pkv
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         t0.record(stream)
         for i in range(steps):
+            v = i % w.num_steps
             r.q.copy_(hq, non_blocking=True)
             r.k.copy_(hk, non_blocking=True)
             r.v.copy_(hv, non_blocking=True)
-            sl_dev.copy_(hsl[i % w.num_steps], non_blocking=True)
-            for l in range(w.num_layers):
-                pkv.append(r.pool, r.bt, sl_dev, r.k[l], r.v[l], l, stream=stream)
-                pkv.decode(r.q[l], r.pool, r.bt, sl_dev, l, w.scale, out=r.out[l],
-                           workspace=r.ws, kernel=r.kernel, stream=stream)
+            r.seq_lens[v].copy_(hsl[v], non_blocking=True)
+            r.replay(i)
             hout.copy_(r.out, non_blocking=True)
         t1.record(stream)
     stream.synchronize()
@@ -380,6 +404,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch without programmatic dependent launch")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -88,6 +88,11 @@ typedef enum {
   PKV_ERR_BAD_SEQ_LEN = -8     /* device: seq_len < 0 (append: < 1) or too long      */
 } pkv_status;
 
+/* Launch flags for pkv_pool_set_launch_flags. */
+#define PKV_LAUNCH_PDL 1          /* programmatic dependent launch (see below) */
+#define PKV_LAUNCH_EARLY_TABLES 2 /* with PDL: decode reads seq_lens and block
+                                     tables before the preceding kernel ends */
+
 /* Decode kernel variants for paged_attention_decode_ex. */
 #define PKV_KERNEL_AUTO 0
 #define PKV_KERNEL_SIMT 1 /* CUDA-core FP32 dot products, warp-shuffle reductions */
@@ -118,6 +123,24 @@ PKV_API void *pkv_pool_data(const pkv_pool *pool);
 PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
 
 /*
+ * Launch options for every later pkv_append / paged_attention_decode call on
+ * this pool.  PKV_LAUNCH_PDL launches the kernels with programmatic stream
+ * serialisation: a kernel may be scheduled while the preceding kernel of the
+ * stream is still running, and waits for it (griddepcontrol.wait) before it
+ * reads or writes any memory, so results are the same as without the flag;
+ * only launch latency is hidden.  Also valid under CUDA graph capture.
+ * PKV_LAUNCH_EARLY_TABLES (only together with PKV_LAUNCH_PDL) lets decode
+ * read seq_lens and the block tables -- never q, the pool or the outputs --
+ * before the preceding kernel of the stream has finished, so its set-up
+ * overlaps that kernel; the caller guarantees that the kernel launched just
+ * before a decode does not write seq_lens or the block tables (an append,
+ * which only reads them, is fine).
+ * flags: 0, PKV_LAUNCH_PDL or PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES, else
+ * PKV_ERR_INVALID_ARG.
+ */
+PKV_API int pkv_pool_set_launch_flags(pkv_pool *pool, int32_t flags);
+
+/*
  * Append (decode step, one token per sequence): for each b with
  * L = seq_lens[b], copy k_new[b][g][:] and v_new[b][g][:] for all 8 kv
  * heads into slot (L-1) % 16 of page block_tables[layer][b][(L-1)/16].
@@ -132,13 +155,11 @@ PKV_API int pkv_append(pkv_pool *pool, const int32_t *block_tables, const int32_
 
 /*
  * Workspace bytes paged_attention_decode needs for this batch on the pool's
- * device (split-KV partial results and merge counters).  The workspace is
- * caller-owned device memory, 256-byte aligned, and must be ZERO-FILLED
- * before its first use.  Every decode that completes puts the part that must
- * start at zero (one merge counter per (sequence, kv head)) back to zero, so
- * the workspace can be reused without clearing it; after a
- * PKV_ERR_DEVICE_TIMEOUT zero it again.  Calls that share one workspace must
- * not overlap in time.
+ * device: the split-KV partial results (m, l and the unnormalised output of
+ * every piece of a split sequence) and the per-sequence split table.  The
+ * workspace is caller-owned device memory, 256-byte aligned; its contents
+ * need no initialisation (every decode writes what it later reads).  Calls
+ * that share one workspace must not overlap in time.
  */
 PKV_API int pkv_decode_workspace_bytes(const pkv_pool *pool, int32_t batch, size_t *bytes_out);
 
@@ -147,8 +168,10 @@ PKV_API int pkv_decode_workspace_bytes(const pkv_pool *pool, int32_t batch, size
  *   out[b][h][:] = sum_{t<L} softmax_t(scale * q[b][h].K[t][h/4]) V[t][h/4]
  * with K/V read in place from the pages block_tables[layer][b][*], FP32
  * online softmax and FP32 accumulation.  Sequences with L == 0 get an
- * all-zero output.  Long contexts are split across the GPU (split-KV) and
- * merged with log-sum-exp weights inside the same launch.  Device errors:
+ * all-zero output.  Long contexts are split across the GPU (split-KV): the
+ * decode kernel writes the pieces to the workspace and a second kernel,
+ * launched right after it on the same stream, merges them with log-sum-exp
+ * weights in a fixed order (results do not depend on timing).  Device errors:
  * L < 0 or L > max_blocks*16 -> PKV_ERR_BAD_SEQ_LEN (that row is written as
  * zeros); a page outside the pool -> PKV_ERR_BAD_PAGE (that page is
  * skipped).  Requires 8 * batch * max_blocks < 2^31.
@@ -164,8 +187,8 @@ PKV_API int paged_attention_decode(const uint16_t *q, const pkv_pool *pool, cons
  *   grid_ctas:   0 = one persistent wave over the device; > 0 = exactly that
  *                many CTAs (the split of long contexts changes with it; the
  *                workspace needed is pkv_decode_workspace_bytes_ex's);
- *   min_chunk:   0 = automatic; > 0 = each warp takes at least this many
- *                (page, kv-head) tiles.
+ *   min_chunk:   0 = automatic; > 0 = each CTA takes at least this many
+ *                pages.
  */
 PKV_API int paged_attention_decode_ex(const uint16_t *q, const pkv_pool *pool,
                               const int32_t *block_tables, const int32_t *seq_lens, int32_t layer,

@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(128) append_kernel(const uint4* __restrict__ k
                                                      const int32_t* __restrict__ seq_lens,
                                                      int32_t* __restrict__ err, int32_t max_blocks,
                                                      int32_t num_pages) {
+  pdl_wait();   // the pool may be in use by the preceding kernel
+  pdl_trigger();
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
   const int kv = tid >> 6;
@@ -87,13 +89,20 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ p
 cudaError_t launch_append(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
                           __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,
                           int32_t* err, int32_t batch, int32_t max_blocks, int32_t num_pages,
-                          cudaStream_t stream) {
+                          int flags, cudaStream_t stream) {
   if (batch == 0) return cudaSuccess;
-  append_kernel<<<batch, 128, 0, stream>>>(reinterpret_cast<const uint4*>(k_new),
-                                           reinterpret_cast<const uint4*>(v_new),
-                                           reinterpret_cast<uint4*>(pool), bt, seq_lens, err,
-                                           max_blocks, num_pages);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(batch);
+  cfg.blockDim = dim3(128);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, append_kernel, reinterpret_cast<const uint4*>(k_new),
+                            reinterpret_cast<const uint4*>(v_new), reinterpret_cast<uint4*>(pool),
+                            bt, seq_lens, err, max_blocks, num_pages);
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,

@@ -9,44 +9,49 @@
 // inferencia de LLM...", section "¿Cómo administra el motor la memoria de la
 // caché KV?").  Decode is memory-bound (same "Construye..." page, section
 // "Prefill vs. Decode"), so the design is about streaming K/V from HBM at
-// full bandwidth with as few instructions per byte as possible.
+// full bandwidth with as few instructions and as little serial latency per
+// byte as possible.
 //
-// Work decomposition (B200 design, not from the pages).  A unit is one
-// (sequence, kv head) pair; its pages form a run of (page, kv head) tiles of
-// 4 KiB (2 KiB of K + 2 KiB of V).  All units' tiles are laid end to end in
-// (sequence, kv head, page) order and the resulting list is cut into equal
-// contiguous ranges, one per warp of a persistent grid (one wave: every SM
-// holds the same number of CTAs).  Each warp is an independent pipeline:
-// lane 0 issues 2-D TMA loads (128-byte swizzle, L2 evict-first, no
-// multicast) of the next tiles into a ring of shared-memory stages guarded
-// by mbarriers, while the whole warp computes on the current tile.  No
-// __syncthreads in the loop.  The 4 query heads of a kv head share every
-// K/V tile load.
+// Work decomposition (B200 design, not from the pages).  Pages are the unit
+// of data movement: a 32 KiB page holds K and V of 16 tokens for all 8 kv
+// heads, and one 2-D TMA box of 256 rows x 128 B (128-byte swizzle, L2
+// evict-first, no multicast) brings a whole page into shared memory.  A CTA
+// has 8 warps, warp g computing kv head g -- the 4 query heads of that group
+// share every K/V tile.  The sequences' pages are laid end to end (each
+// sequence also costs kSeqCost pages of fixed work) and the total is cut into
+// equal contiguous ranges, one per CTA of a persistent grid (one wave, the
+// same number of CTAs on every SM).  Lane 0 of warp 0 is the producer: it
+// walks the CTA's range, reads each page's block-table entry, and issues the
+// page's TMA load -- plus, for a page that starts a sequence, a bulk copy of
+// the sequence's 32 query rows -- into a ring of stages, each guarded by a
+// "full" mbarrier (TMA transaction bytes) and an "empty" mbarrier (one
+// arrival per warp once it is done with the stage).
 //
-// A unit that falls inside one warp's range is finished in registers.  A
-// unit cut by range boundaries is split-KV: each piece writes (m, l, acc) to
-// the workspace and the last piece to arrive (atomic counter per unit)
-// merges them in a fixed order with log-sum-exp weights and writes out, so
-// the split needs no second launch and the result does not depend on which
-// warp finishes last.  Every lane works in log2 units: scores are scaled by
-// scale * log2(e) and exponentials are exp2.
+// A sequence whose pages all fall in one CTA is finished in registers.  A
+// sequence cut by range boundaries is split-KV: each piece writes (m, l, acc)
+// per kv head to the workspace and the last piece to arrive (atomic counter
+// per (sequence, kv head)) merges them in a fixed order with log-sum-exp
+// weights and writes out, so the split needs no second launch and the result
+// does not depend on which CTA finishes last.  Scores are kept in log2 units
+// (scaled by scale * log2(e)) and exponentials are exp2.
+//
+// Two compute variants share this skeleton:
+//  - SimtCompute: CUDA-core FP32 dot products (packed FFMA2) with
+//    warp-shuffle reductions for the dot products, the max and the sum;
+//  - MmaCompute: the 16-token x 4-head tile on the tensor cores
+//    (mma.sync m16n8k16, BF16 in, FP32 accumulate) for both Q.K^T and P.V,
+//    with P split into two BF16 terms (hi + lo) so that rounding P to BF16
+//    costs no accuracy; softmax stays FP32 on the CUDA cores.
 #include "pkv_internal.cuh"
 
 namespace pkv {
 
-constexpr int kWarps = 4;                       // warps per CTA
-constexpr int kStages = 4;                      // tiles in flight per warp
-constexpr int kStageBytes = 2 * kTileBytes;     // K tile + V tile
 constexpr unsigned kFull = 0xFFFFFFFFu;
-
-constexpr size_t kTilesBytes = size_t(kWarps) * kStages * kStageBytes;
-constexpr size_t kBarsOff = kTilesBytes;
-constexpr size_t kLensOff = kBarsOff + size_t(kWarps) * kStages * 8;
-
-static size_t decode_smem_bytes(int32_t batch) {
-  // tiles, mbarriers, lengths [B], page-count prefix [B+1], alignment slack
-  return kLensOff + size_t(batch) * 4 + size_t(batch + 1) * 4 + 1024;
-}
+constexpr int kWarps = kKvHeads;                    // one warp per kv head
+constexpr int kPageBytes = 2 * kKvHeads * kTileBytes;  // 32 KiB
+constexpr int kQRowsBytes = kQHeads * kRowBytes;    // a sequence's 32 query rows: 4 KiB
+constexpr int kStageBytes = kPageBytes + kQRowsBytes;
+constexpr int kScratchBytes = 512;                  // per-warp P^T transpose buffer
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -68,16 +73,19 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // only when a unit ends.
 // ---------------------------------------------------------------------------
 struct SimtCompute {
+  static constexpr int kStages = 3;
+  static constexpr int kMinBlocks = 1;
+
   float2 q2[kGroup][4];   // q[h][8c + 2e], q[h][8c + 2e + 1]
   float2 acc[kGroup][4];  // sum over this lane's tokens of p * v[8c + 2e ..]
   float m[kGroup];        // running max per head (log2 units), warp-uniform
   float lsum[2];          // sum of p over this lane's scores, heads 2*b2 + k
 
-  __device__ __forceinline__ void begin(const __nv_bfloat16* qrows, int lane) {
+  __device__ __forceinline__ void begin(uint32_t qslot, int lane) {
     const int c = lane & 7;
 #pragma unroll
     for (int h = 0; h < kGroup; ++h) {
-      const uint4 w = *reinterpret_cast<const uint4*>(qrows + h * kDim + 8 * c);
+      const uint4 w = lds128(qslot + h * kRowBytes + 16 * c);
       q2[h][0] = bf16x2_to_float2(w.x);
       q2[h][1] = bf16x2_to_float2(w.y);
       q2[h][2] = bf16x2_to_float2(w.z);
@@ -89,8 +97,8 @@ struct SimtCompute {
     lsum[0] = lsum[1] = 0.f;
   }
 
-  __device__ __forceinline__ void consume(uint32_t ktile, uint32_t vtile, int nvalid,
-                                          float scale_log2, int lane) {
+  __device__ __forceinline__ void consume(uint32_t ktile, uint32_t vtile, uint32_t /*scratch*/,
+                                          int nvalid, float scale_log2, int lane) {
     const int c = lane & 7, tg = lane >> 3;
     const int b0 = c & 1, b1 = (c >> 1) & 1, b2 = c >> 2;
 
@@ -262,12 +270,179 @@ struct SimtCompute {
 };
 
 // ---------------------------------------------------------------------------
+// Tensor-core compute (mma.sync m16n8k16, BF16 x BF16 -> FP32).
+//
+// Lane = (r = lane / 4, qd = lane % 4), the mma fragment coordinates.
+//  QK:  S^T[t][h] = sum_d K[t][d] Q[h][d]: M = 16 tokens (A = the K tile,
+//       ldmatrix from the swizzled stage), N = 8 (4 real heads + 4 zero
+//       columns), K = 64 in 4 steps.  Products of BF16 values are exact in
+//       FP32, so this is the same arithmetic as the CUDA-core dot product.
+//       Lane holds S^T[r][2qd..2qd+1] and S^T[r+8][2qd..2qd+1].
+//  softmax: FP32, per head over the 16 tokens (2 per lane x 8 lanes).
+//  PV:  O^T[d][h] = sum_t V^T[d][t] P^T[t][h]: M = 64 dims in 4 tiles
+//       (A = V^T via ldmatrix.trans), N = 8 heads, K = 16 tokens.  P^T is
+//       written to a per-warp scratch in [t][h] order and read back with
+//       ldmatrix.trans as the B fragment.  P is split into
+//       hi = bf16(p) and lo = bf16(p - hi), two MMAs, so the product keeps
+//       ~16 mantissa bits of p.
+//  Lane holds O^T[16mt + r (+8)][2qd..2qd+1]: its softmax heads and its
+//  accumulator heads are the same, so rescaling needs no data movement.
+// ---------------------------------------------------------------------------
+struct MmaCompute {
+  static constexpr int kStages = 2;
+  static constexpr int kMinBlocks = 2;
+
+  uint32_t qb[4][2];  // B fragments of Q^T, k-steps 0..3 (zero for lanes with r >= 4)
+  float o[4][4];      // O^T accumulators, m-tiles 0..3
+  float m[2];         // running max of heads 2qd, 2qd+1 (log2 units)
+  float l[2];         // this lane's share of the softmax denominators
+
+  __device__ __forceinline__ void begin(uint32_t qslot, int lane) {
+    const int r = lane >> 2, qd = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      if (r < kGroup) {
+        const uint32_t a = qslot + r * kRowBytes + (16 * ks + 2 * qd) * 2;
+        qb[ks][0] = lds32(a);
+        qb[ks][1] = lds32(a + 16);
+      } else {
+        qb[ks][0] = qb[ks][1] = 0u;
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
+  }
+
+  __device__ __forceinline__ void consume(uint32_t ktile, uint32_t vtile, uint32_t scratch,
+                                          int nvalid, float scale_log2, int lane) {
+    const int r = lane >> 2, qd = lane & 3;
+    // ---- S^T = K Q^T
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(a, ktile + swz(lane & 15, 2 * ks + (lane >> 4)));
+      mma_bf16_16816(s, a, qb[ks][0], qb[ks][1]);
+    }
+    // ---- FP32 online softmax; tokens r and r + 8, heads 2qd and 2qd + 1
+    const bool v0 = r < nvalid, v1 = r + 8 < nvalid;
+    const float x0 = v0 ? s[0] * scale_log2 : -INFINITY;
+    const float x1 = v0 ? s[1] * scale_log2 : -INFINITY;
+    const float x2 = v1 ? s[2] * scale_log2 : -INFINITY;
+    const float x3 = v1 ? s[3] * scale_log2 : -INFINITY;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+    }
+    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+    const float a0 = fast_exp2(m[0] - mn0), a1 = fast_exp2(m[1] - mn1);
+    m[0] = mn0;
+    m[1] = mn1;
+    const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
+    const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
+    l[0] = fmaf(l[0], a0, p0 + p2);
+    l[1] = fmaf(l[1], a1, p1 + p3);
+    // ---- P^T, split into BF16 hi + lo, through the scratch ([t][8 heads])
+    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+    const uint32_t l01 = pack_bf16x2(p0 - __uint_as_float(h01 << 16),
+                                     p1 - __uint_as_float(h01 & 0xFFFF0000u));
+    const uint32_t l23 = pack_bf16x2(p2 - __uint_as_float(h23 << 16),
+                                     p3 - __uint_as_float(h23 & 0xFFFF0000u));
+    __syncwarp();   // previous tile's scratch reads are done
+    const uint32_t w0 = scratch + r * 16 + qd * 4;
+    sts32(w0, h01);
+    sts32(w0 + 128, h23);
+    sts32(w0 + 256, l01);
+    sts32(w0 + 384, l23);
+    __syncwarp();
+    uint32_t pb[4];   // hi: b0, b1; lo: b0, b1
+    ldsm_x4_trans(pb, scratch + (lane >> 3) * 128 + (lane & 7) * 16);
+    // ---- rescale and O^T += V^T P^T (hi, lo)
+    uint32_t mlo = kFull, mhi = kFull;
+    if (nvalid < kTokens) {   // zero V rows past the context: 0 * NaN would be NaN
+      const int t = 2 * qd;
+      mlo = (t < nvalid ? 0x0000FFFFu : 0u) | (t + 1 < nvalid ? 0xFFFF0000u : 0u);
+      mhi = (t + 8 < nvalid ? 0x0000FFFFu : 0u) | (t + 9 < nvalid ? 0xFFFF0000u : 0u);
+    }
+    const int vrow = (lane & 7) + ((lane >> 4) << 3);
+    const int vchunk = (lane >> 3) & 1;
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_trans(a, vtile + swz(vrow, 2 * mt + vchunk));
+      a[0] &= mlo;
+      a[1] &= mlo;
+      a[2] &= mhi;
+      a[3] &= mhi;
+      o[mt][0] *= a0;
+      o[mt][1] *= a1;
+      o[mt][2] *= a0;
+      o[mt][3] *= a1;
+      mma_bf16_16816(o[mt], a, pb[0], pb[1]);
+      mma_bf16_16816(o[mt], a, pb[2], pb[3]);
+    }
+  }
+
+  // Full softmax denominators of heads 2qd, 2qd + 1.
+  __device__ __forceinline__ void reduce_l(float& l0, float& l1) const {
+    l0 = l[0];
+    l1 = l[1];
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(kFull, l0, off);
+      l1 += __shfl_xor_sync(kFull, l1, off);
+    }
+  }
+
+  __device__ __forceinline__ void write_rows(float* rows, int lane, float s0, float s1) const {
+    const int r = lane >> 2, qd = lane & 3;
+    if (qd < 2) {
+      float* h0 = rows + (2 * qd) * kDim + r;
+      float* h1 = h0 + kDim;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        h0[16 * mt] = o[mt][0] * s0;
+        h1[16 * mt] = o[mt][1] * s1;
+        h0[16 * mt + 8] = o[mt][2] * s0;
+        h1[16 * mt + 8] = o[mt][3] * s1;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void finalize(float* out_rows, int lane) const {
+    float l0, l1;
+    reduce_l(l0, l1);
+    write_rows(out_rows, lane, 1.f / l0, 1.f / l1);
+  }
+
+  __device__ __forceinline__ void store_partial(float* P, int lane) const {
+    float l0, l1;
+    reduce_l(l0, l1);
+    const int qd = lane & 3;
+    if (lane < 2) {   // r == 0, qd == lane
+      P[2 * qd] = m[0];
+      P[2 * qd + 1] = m[1];
+      P[kGroup + 2 * qd] = l0;
+      P[kGroup + 2 * qd + 1] = l1;
+    }
+    write_rows(P + 2 * kGroup, lane, 1.f, 1.f);
+  }
+};
+
+
+// ---------------------------------------------------------------------------
 // Shared pieces of the persistent kernel
 // ---------------------------------------------------------------------------
 
-// Lengths of all sequences and the exclusive prefix of their page counts,
-// computed by every CTA (B integers from L2; cheaper than a second launch).
-// Invalid lengths count as empty sequences and are reported.
+// Lengths of all sequences and the prefix of their page counts, computed by
+// every CTA (B integers from L2; cheaper than a second launch).  Invalid
+// lengths count as empty sequences and are reported.
 __device__ __forceinline__ void cta_lengths(const DecodeArgs& a, int32_t* s_len, int32_t* s_pfx,
                                             int32_t* s_tot) {
   const int B = a.batch, tid = threadIdx.x, nthr = blockDim.x;
@@ -300,22 +475,35 @@ __device__ __forceinline__ void cta_lengths(const DecodeArgs& a, int32_t* s_len,
     run += (s_len[b] + kTokens - 1) / kTokens;
     s_pfx[b + 1] = run;
   }
-  __syncthreads();
 }
 
-// (sequence, kv head, page) of flat tile index f < 8 * s_pfx[B].
-__device__ __forceinline__ void locate(const int32_t* s_pfx, int B, int32_t f, int& b, int& g,
-                                       int& j) {
+// Cost position where sequence b starts: every sequence costs its pages plus
+// kSeqCost.  Page j of sequence b sits at seq_cost(b) + kSeqCost + j.
+__device__ __forceinline__ int64_t seq_cost(const int32_t* s_pfx, int b) {
+  return static_cast<int64_t>(s_pfx[b]) + static_cast<int64_t>(kSeqCost) * b;
+}
+
+// Number of pages whose cost position is below x.
+__device__ __forceinline__ int32_t pages_below(const int32_t* s_pfx, int B, int64_t x) {
+  if (x >= seq_cost(s_pfx, B)) return s_pfx[B];
   int lo = 0, hi = B - 1;
-  while (lo < hi) {   // largest b with 8 * pfx[b] <= f
+  while (lo < hi) {   // largest b with seq_cost(b) <= x
     const int mid = (lo + hi + 1) >> 1;
-    if (kKvHeads * s_pfx[mid] <= f) lo = mid; else hi = mid - 1;
+    if (seq_cost(s_pfx, mid) <= x) lo = mid; else hi = mid - 1;
+  }
+  const int64_t off = x - seq_cost(s_pfx, lo) - kSeqCost;
+  return s_pfx[lo] + static_cast<int32_t>(off < 0 ? 0 : off);
+}
+
+// (sequence, page) of flat page index f < s_pfx[B].
+__device__ __forceinline__ void locate(const int32_t* s_pfx, int B, int32_t f, int& b, int& j) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {   // largest b with pfx[b] <= f
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_pfx[mid] <= f) lo = mid; else hi = mid - 1;
   }
   b = lo;
-  const int np = s_pfx[b + 1] - s_pfx[b];
-  const int rel = f - kKvHeads * s_pfx[b];
-  g = rel / np;
-  j = rel - g * np;
+  j = f - s_pfx[b];
 }
 
 __device__ __forceinline__ void zero_rows(float* rows, int lane) {
@@ -324,9 +512,31 @@ __device__ __forceinline__ void zero_rows(float* rows, int lane) {
   for (int i = lane; i < kQHeads * kDim / 4; i += 32) d[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// Fixed-order log-sum-exp merge of `cnt` partial records.  Lane handles dims
-// 2*lane, 2*lane+1 of all 4 heads.
-__device__ __noinline__ void merge_partials(const float* P, int cnt, float* out_rows, int lane) {
+// Fixed-order log-sum-exp merge of `cnt` partial records P[0], P[stride],
+// ... (pieces of one (sequence, kv head) unit, in piece order):
+//   M[h] = max_s m_s[h],  w_s[h] = exp2(m_s[h] - M[h]),
+//   S[h] = sum_s w_s[h] l_s[h],  O[h][d] = sum_s w_s[h] acc_s[h][d].
+// With `final`, out[h][d] = O / S (zero where S == 0); otherwise (M, S, O)
+// is written as one partial record at `out`.  Pieces are taken 32 at a time
+// (running max rescaled between groups, a fixed order): lane s reads m and l
+// of piece s, and every lane accumulates dims 2*lane, 2*lane+1 of the 4 heads
+// with the loads of kMergeBatch pieces in flight.  kShared: P lives in shared
+// memory (plain loads) instead of global memory (L2 loads).
+constexpr int kMergeBatch = 8;
+
+template <bool kShared>
+__device__ __forceinline__ float4 ld4(const float* p) {
+  return kShared ? *reinterpret_cast<const float4*>(p) : __ldcg(reinterpret_cast<const float4*>(p));
+}
+template <bool kShared>
+__device__ __forceinline__ float2 ld2(const float* p) {
+  return kShared ? *reinterpret_cast<const float2*>(p) : __ldcg(reinterpret_cast<const float2*>(p));
+}
+
+template <bool kShared>
+__device__ __forceinline__ void merge_partials(const float* P, int cnt, int stride, float* out,
+                                               bool final, int lane) {
+  const int64_t step = static_cast<int64_t>(stride) * kPartialFloats;
   float M[kGroup], S[kGroup];
   float2 O[kGroup];
 #pragma unroll
@@ -335,201 +545,329 @@ __device__ __noinline__ void merge_partials(const float* P, int cnt, float* out_
     S[h] = 0.f;
     O[h] = make_float2(0.f, 0.f);
   }
-#pragma unroll 2
-  for (int s = 0; s < cnt; ++s) {
-    const float* p = P + static_cast<int64_t>(s) * kPartialFloats;
-    const float4 m4 = __ldcg(reinterpret_cast<const float4*>(p));
-    const float4 l4 = __ldcg(reinterpret_cast<const float4*>(p) + 1);
-    const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-    const float ll[4] = {l4.x, l4.y, l4.z, l4.w};
+  for (int s0 = 0; s0 < cnt; s0 += 32) {
+    const int n = min(32, cnt - s0);
+    float mm[kGroup] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    float ll[kGroup] = {0.f, 0.f, 0.f, 0.f};
+    if (lane < n) {
+      const float* p = P + (s0 + lane) * step;
+      const float4 m4 = ld4<kShared>(p), l4 = ld4<kShared>(p + 4);
+      mm[0] = m4.x; mm[1] = m4.y; mm[2] = m4.z; mm[3] = m4.w;
+      ll[0] = l4.x; ll[1] = l4.y; ll[2] = l4.z; ll[3] = l4.w;
+    }
+    float wgt[kGroup];
 #pragma unroll
     for (int h = 0; h < kGroup; ++h) {
-      const float2 o = __ldcg(reinterpret_cast<const float2*>(p + 2 * kGroup + h * kDim) + lane);
-      const float mn = fmaxf(M[h], mm[h]);
-      if (mn == -INFINITY) continue;   // nothing accumulated on either side yet
-      const float sa = fast_exp2(M[h] - mn), sb = fast_exp2(mm[h] - mn);
-      S[h] = S[h] * sa + ll[h] * sb;
-      O[h].x = O[h].x * sa + o.x * sb;
-      O[h].y = O[h].y * sa + o.y * sb;
+      float mc = mm[h];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) mc = fmaxf(mc, __shfl_xor_sync(kFull, mc, off));
+      const float mn = fmaxf(M[h], mc);
+      if (mn != -INFINITY) {   // rescale what was accumulated under the old max
+        const float r = fast_exp2(M[h] - mn);
+        S[h] *= r;
+        O[h].x *= r;
+        O[h].y *= r;
+      }
       M[h] = mn;
+      // a piece whose pages were all skipped has m = -inf and weight 0
+      wgt[h] = (mm[h] == -INFINITY) ? 0.f : fast_exp2(mm[h] - mn);
+      S[h] = fmaf(wgt[h], ll[h], S[h]);
+    }
+    const float* base = P + s0 * step + 2 * kGroup;
+    for (int k0 = 0; k0 < n; k0 += kMergeBatch) {
+      float2 v[kMergeBatch][kGroup];
+#pragma unroll
+      for (int kk = 0; kk < kMergeBatch; ++kk)
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h)
+          v[kk][h] = (k0 + kk < n) ? ld2<kShared>(base + (k0 + kk) * step + h * kDim + 2 * lane)
+                                   : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int kk = 0; kk < kMergeBatch; ++kk)
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) {
+          const float wk = __shfl_sync(kFull, wgt[h], (k0 + kk) & 31);
+          O[h].x = fmaf(wk, v[kk][h].x, O[h].x);
+          O[h].y = fmaf(wk, v[kk][h].y, O[h].y);
+        }
     }
   }
 #pragma unroll
-  for (int h = 0; h < kGroup; ++h) {
-    const float inv = S[h] > 0.f ? 1.f / S[h] : 0.f;
-    reinterpret_cast<float2*>(out_rows + h * kDim)[lane] = make_float2(O[h].x * inv, O[h].y * inv);
+  for (int h = 0; h < kGroup; ++h)
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) S[h] += __shfl_xor_sync(kFull, S[h], off);
+  if (final) {
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h) {
+      const float inv = S[h] > 0.f ? 1.f / S[h] : 0.f;
+      reinterpret_cast<float2*>(out + h * kDim)[lane] = make_float2(O[h].x * inv, O[h].y * inv);
+    }
+  } else {
+    if (lane == 0) {
+      reinterpret_cast<float4*>(out)[0] = make_float4(M[0], M[1], M[2], M[3]);
+      reinterpret_cast<float4*>(out)[1] = make_float4(S[0], S[1], S[2], S[3]);
+    }
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h)
+      reinterpret_cast<float2*>(out + 2 * kGroup + h * kDim)[lane] = O[h];
   }
 }
 
-// End of a unit's piece inside this warp's range: finish it in registers, or
-// hand it to the split-KV merge.
+// Split-KV bookkeeping of sequence b: the CTA range of its first page and
+// its number of pieces (CTAs its pages span).  Partial records live at
+// [g][b + cta], so the pieces of one (sequence, kv head) unit are the
+// consecutive slots S0 .. S0 + K - 1 with S0 = g * (B + grid) + b + c_first
+// (b + cta is distinct for every piece of head g because both only grow
+// along the page order).
+__device__ __forceinline__ int2 split_of(const int32_t* s_pfx, int b, int64_t chunk) {
+  const int np = s_pfx[b + 1] - s_pfx[b];
+  if (np == 0) return make_int2(0, 0);
+  const int64_t first = seq_cost(s_pfx, b) + kSeqCost;
+  const int c_first = static_cast<int>(first / chunk);
+  return make_int2(c_first, static_cast<int>((first + np - 1) / chunk) - c_first + 1);
+}
+
+// End of a sequence's piece inside this CTA's range, for kv head g (= this
+// warp): finish it in registers when the CTA holds the whole sequence, else
+// store the piece for the merge kernel that follows.
 template <class C>
 __device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a,
                                            const int32_t* s_pfx, int b, int g, int j0, int j1,
-                                           int np, int w, int64_t chunk, int lane) {
-  float* out_rows = a.out + (static_cast<int64_t>(b) * kQHeads + g * kGroup) * kDim;
+                                           int np, int64_t chunk, int lane) {
   if (j0 == 0 && j1 == np - 1) {
-    cmp.finalize(out_rows, lane);
+    cmp.finalize(a.out + (static_cast<int64_t>(b) * kQHeads + g * kGroup) * kDim, lane);
     return;
   }
-  const int u = b * kKvHeads + g;
-  const int64_t start = static_cast<int64_t>(kKvHeads) * s_pfx[b] + static_cast<int64_t>(g) * np;
-  const int w_first = static_cast<int>(start / chunk);
-  const int w_last = static_cast<int>((start + np - 1) / chunk);
-  cmp.store_partial(a.partials + static_cast<int64_t>(u + w) * kPartialFloats, lane);
-  __threadfence();
-  __syncwarp();
-  int prev = 0;
-  if (lane == 0) prev = atomicAdd(a.counters + u, 1);
-  prev = __shfl_sync(kFull, prev, 0);
-  if (prev != w_last - w_first) return;   // not the last piece of this unit
-  __threadfence();
-  merge_partials(a.partials + static_cast<int64_t>(u + w_first) * kPartialFloats,
-                 w_last - w_first + 1, out_rows, lane);
-  if (lane == 0) a.counters[u] = 0;       // ready for the next launch
+  const int2 sp = split_of(s_pfx, b, chunk);
+  const int64_t slot = static_cast<int64_t>(g) * (a.batch + gridDim.x) + b + blockIdx.x;
+  cmp.store_partial(a.partials + slot * kPartialFloats, lane);
+  (void)sp;
 }
 
-// Producer-side description of 32 consecutive tiles: lane i -> tile f0 + i.
-__device__ __forceinline__ void load_tile_batch(const DecodeArgs& a, const int32_t* s_pfx,
-                                                int32_t f, int32_t f_end, int32_t& phys,
-                                                int32_t& kvh) {
+// Producer-side description of page f (this lane's slot of a 32-page batch):
+// physical page, and (sequence << 1) | starts-a-sequence-in-this-range.
+__device__ __forceinline__ void load_page_batch(const DecodeArgs& a, const int32_t* s_pfx,
+                                                int32_t f, int32_t f_begin, int32_t f_end,
+                                                int32_t& phys, int32_t& info) {
   phys = -1;
-  kvh = 0;
+  info = 0;
   if (f < f_end) {
-    int b, g, j;
-    locate(s_pfx, a.batch, f, b, g, j);
+    int b, j;
+    locate(s_pfx, a.batch, f, b, j);
     phys = __ldg(a.bt + static_cast<int64_t>(b) * a.max_blocks + j);
-    kvh = g;
+    info = (b << 1) | ((j == 0 || f == f_begin) ? 1 : 0);
   }
 }
 
 template <class C>
-__global__ void __launch_bounds__(kWarps * 32, 3)
+struct SmemPlan {
+  static constexpr int S = C::kStages;
+  static constexpr size_t stages = 0;   // [S][page 32 KiB | query rows 4 KiB]
+  static constexpr size_t scratch = stages + size_t(S) * kStageBytes;
+  static constexpr size_t full = scratch + size_t(kWarps) * kScratchBytes;
+  static constexpr size_t empty = full + size_t(S) * 8;
+  static constexpr size_t flags = empty + size_t(S) * 8;   // [S] bad page, [1] abort
+  static constexpr size_t tot = flags + size_t(S + 1) * 4;  // [kWarps] scan totals
+  static constexpr size_t lens = tot + size_t(kWarps) * 4;
+  static size_t bytes(int32_t batch) {
+    // lengths [B] and page-count prefix [B+1], plus 1024 B of alignment slack
+    return lens + size_t(batch) * 4 + size_t(batch + 1) * 4 + 1024;
+  }
+};
+
+template <class C>
+__global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+  constexpr int kS = C::kStages;
+  using L = SmemPlan<C>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int32_t s_tot[kWarps];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = a.batch;
-  int32_t* s_len = reinterpret_cast<int32_t*>(smem + kLensOff);
+  volatile int32_t* s_flags = reinterpret_cast<int32_t*>(smem + L::flags);
+  int32_t* s_len = reinterpret_cast<int32_t*>(smem + L::lens);
   int32_t* s_pfx = s_len + B;
+  const uint32_t base = smem_addr(smem);
+  const uint32_t full = base + L::full, empty = base + L::empty;
+  const uint32_t scratch = base + L::scratch + warp * kScratchBytes;
 
-  cta_lengths(a, s_len, s_pfx, s_tot);
-
-  const uint32_t tiles = smem_addr(smem) + warp * kStages * kStageBytes;
-  const uint32_t bars = smem_addr(smem + kBarsOff) + warp * kStages * 8;
-  if (lane == 0) {
+  if (threadIdx.x == 0) {
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) mbar_init(bars + 8 * s, 1);
+    for (int s = 0; s < kS; ++s) {
+      mbar_init(full + 8 * s, 1);
+      mbar_init(empty + 8 * s, kWarps);
+      s_flags[s] = 0;
+    }
+    s_flags[kS] = 0;
     fence_mbar_init();
   }
-  __syncwarp();
+  // With kLaunchEarlyTables the lengths and block tables are read before the
+  // preceding kernel of the stream has finished (the caller guarantees that
+  // kernel does not write them); q, the pool and the outputs only after.
+  const bool early = (a.flags & kLaunchEarlyTables) != 0;
+  if (!early) pdl_wait();
+  pdl_trigger();
+  cta_lengths(a, s_len, s_pfx, reinterpret_cast<int32_t*>(smem + L::tot));
+  __syncthreads();
 
-  const int W = gridDim.x * kWarps;
-  const int w = blockIdx.x * kWarps + warp;
-  const int32_t P = kKvHeads * s_pfx[B];
-  int64_t chunk = (static_cast<int64_t>(P) + W - 1) / W;
+  const int G = gridDim.x;
+  const int64_t total = seq_cost(s_pfx, B);
+  int64_t chunk = (total + G - 1) / G;
   if (chunk < a.min_chunk) chunk = a.min_chunk;
   if (chunk < 1) chunk = 1;
+  const int64_t x0 = static_cast<int64_t>(blockIdx.x) * chunk;
+  const int32_t p0 = x0 < total ? pages_below(s_pfx, B, x0) : 0;
+  const int32_t p1 = x0 < total ? pages_below(s_pfx, B, x0 + chunk) : 0;
+  const int n = p1 - p0;
 
-  for (int b = w; b < B; b += W)
-    if (s_pfx[b + 1] == s_pfx[b]) zero_rows(a.out + static_cast<int64_t>(b) * kQHeads * kDim, lane);
-
-  const int64_t q0l = static_cast<int64_t>(w) * chunk;
-  if (q0l >= P) return;
-  const int32_t q0 = static_cast<int32_t>(q0l);
-  const int32_t q1 = static_cast<int32_t>(q0l + chunk < P ? q0l + chunk : P);
-  const int n = q1 - q0;
-  const uint64_t policy = l2_evict_first_policy();
-
-  // producer state: tile descriptions for batches k (cur) and k + 1 (nxt)
-  int32_t cur_phys, cur_g, nxt_phys, nxt_g;
-  load_tile_batch(a, s_pfx, q0 + lane, q1, cur_phys, cur_g);
-  load_tile_batch(a, s_pfx, q0 + 32 + lane, q1, nxt_phys, nxt_g);
+  // ---- producer (warp 0): page descriptions for batches k (cur), k+1 (nxt)
+  int32_t cur_phys = -1, cur_info = 0, nxt_phys = -1, nxt_info = 0;
   int cur_k = 0;
-  uint32_t bad = 0;   // bit s set: stage s holds a skipped (invalid) page
-  int prod = 0;
+  uint64_t policy = 0;
+  if (warp == 0 && n > 0) {
+    policy = l2_evict_first_policy();
+    load_page_batch(a, s_pfx, p0 + lane, p0, p1, cur_phys, cur_info);
+    load_page_batch(a, s_pfx, p0 + 32 + lane, p0, p1, nxt_phys, nxt_info);
+  }
+  if (early) pdl_wait();
 
+  // every sequence once across the grid: its split for the merge kernel, and
+  // zero output rows if it is empty
+  for (int b = blockIdx.x * kWarps + warp; b < B; b += G * kWarps) {
+    const int2 sp = split_of(s_pfx, b, chunk);
+    if (lane == 0) a.meta[b] = sp;
+    if (sp.y == 0) zero_rows(a.out + static_cast<int64_t>(b) * kQHeads * kDim, lane);
+  }
+  if (n <= 0) return;
+  // Issue page r into stage r % kS (warp 0 only; stage known to be free).
   auto issue = [&](int r) {
     if ((r >> 5) != cur_k) {
       cur_phys = nxt_phys;
-      cur_g = nxt_g;
+      cur_info = nxt_info;
       ++cur_k;
-      load_tile_batch(a, s_pfx, q0 + 32 * (cur_k + 1) + lane, q1, nxt_phys, nxt_g);
+      load_page_batch(a, s_pfx, p0 + 32 * (cur_k + 1) + lane, p0, p1, nxt_phys, nxt_info);
     }
     const int32_t phys = __shfl_sync(kFull, cur_phys, r & 31);
-    const int32_t g = __shfl_sync(kFull, cur_g, r & 31);
-    const int st = r % kStages;
-    const bool ok = static_cast<uint32_t>(phys) < static_cast<uint32_t>(a.num_pages);
+    const int32_t info = __shfl_sync(kFull, cur_info, r & 31);
     if (lane == 0) {
-      const uint32_t bar = bars + 8 * st;
-      if (ok) {
-        mbar_arrive_expect_tx(bar, kStageBytes);
-        const int32_t y = phys * kRowsPerPage + g * kTokens;
-        tma_load_tile(tiles + st * kStageBytes, &tmap, 0, y, bar, policy);
-        tma_load_tile(tiles + st * kStageBytes + kTileBytes, &tmap, 0, y + kKvHeads * kTokens, bar,
-                      policy);
+      const int st = r % kS;
+      const uint32_t bar = full + 8 * st;
+      const uint32_t dst = base + L::stages + st * kStageBytes;
+      const bool ok = static_cast<uint32_t>(phys) < static_cast<uint32_t>(a.num_pages);
+      const bool start = info & 1;
+      s_flags[st] = ok ? 0 : 1;
+      if (!ok) record_error(a.err, kErrBadPage);
+      const uint32_t bytes = (ok ? kPageBytes : 0) + (start ? kQRowsBytes : 0);
+      if (bytes) {
+        mbar_arrive_expect_tx(bar, bytes);
+        if (ok) tma_load_tile(dst, &tmap, 0, phys * kRowsPerPage, bar, policy);
+        if (start)
+          bulk_load(dst + kPageBytes, a.q + static_cast<int64_t>(info >> 1) * kQHeads * kDim,
+                    kQRowsBytes, bar);
       } else {
-        record_error(a.err, kErrBadPage);
         mbar_arrive(bar);
       }
     }
-    bad = ok ? (bad & ~(1u << st)) : (bad | (1u << st));
   };
+  if (warp == 0)
+    for (int r = 0; r < n && r < kS; ++r) issue(r);
 
-  // consumer state
-  int b, g, j;
-  locate(s_pfx, B, q0, b, g, j);
+  // ---- consumers (all 8 warps; warp g computes kv head g)
+  int b, j;
+  locate(s_pfx, B, p0, b, j);
   int np = s_pfx[b + 1] - s_pfx[b];
-  int L = s_len[b];
+  int Lb = s_len[b];
   int j_first = j;
+  bool need_q = true;
   C cmp;
-  cmp.begin(a.q + (static_cast<int64_t>(b) * kQHeads + g * kGroup) * kDim, lane);
-
-  for (; prod < n && prod < kStages; ++prod) issue(prod);
 
   for (int r = 0; r < n; ++r) {
-    const int st = r % kStages;
-    const uint32_t parity = static_cast<uint32_t>(r / kStages) & 1u;
-    if (!mbar_try_wait(bars + 8 * st, parity) && !mbar_wait_bounded(bars + 8 * st, parity)) {
-      // A copy never landed.  Record it, wait (bounded) for the other copies
-      // this warp still has in flight, and stop; the workspace counters of
-      // this launch are then unreliable and must be zeroed again.
+    const int st = r % kS;
+    if (warp == 0 && r >= 1 && r - 1 + kS < n) {
+      // refill the stage that page r - 1 used, once every warp released it
+      const int rr = r - 1;
+      const uint32_t eb = empty + 8 * (rr % kS);
+      const uint32_t par = static_cast<uint32_t>(rr / kS) & 1u;
+      if (!mbar_try_wait(eb, par) && !mbar_wait_bounded(eb, par)) {
+        if (lane == 0) record_error(a.err, kErrTimeout);
+        s_flags[kS] = 1;
+        // copies already issued land in stages r-1+1 .. r-2+kS; wait for them
+        for (int k = r; k < r - 1 + kS && k < n; ++k)
+          mbar_wait_bounded(full + 8 * (k % kS), static_cast<uint32_t>(k / kS) & 1u);
+        return;
+      }
+      issue(rr + kS);
+    }
+    const uint32_t fb = full + 8 * st;
+    const uint32_t par = static_cast<uint32_t>(r / kS) & 1u;
+    if (!mbar_try_wait(fb, par) && !mbar_wait_bounded(fb, par)) {
       if (lane == 0) record_error(a.err, kErrTimeout);
-      for (int rr = r + 1; rr < prod; ++rr)
-        mbar_wait_bounded(bars + 8 * (rr % kStages), static_cast<uint32_t>(rr / kStages) & 1u);
+      s_flags[kS] = 1;
       return;
     }
-    if (!((bad >> st) & 1u)) {
-      const int nvalid = min(kTokens, L - kTokens * j);
-      cmp.consume(tiles + st * kStageBytes, tiles + st * kStageBytes + kTileBytes, nvalid,
-                  a.scale_log2, lane);
+    if (s_flags[kS]) return;   // another warp gave up; results are void
+    const uint32_t stage = base + L::stages + st * kStageBytes;
+    if (need_q) {
+      cmp.begin(stage + kPageBytes + warp * (kGroup * kRowBytes), lane);
+      need_q = false;
+    }
+    if (!s_flags[st]) {
+      const int nvalid = min(kTokens, Lb - kTokens * j);
+      const uint32_t ktile = stage + warp * kTileBytes;
+      cmp.consume(ktile, ktile + kKvHeads * kTileBytes, scratch, nvalid, a.scale_log2, lane);
     }
     __syncwarp();
-    if (prod < n) {
-      issue(prod);
-      ++prod;
-    }
+    if (lane == 0) mbar_arrive(empty + 8 * st);
     if (j == np - 1 || r == n - 1) {
-      flush_unit(cmp, a, s_pfx, b, g, j_first, j, np, w, chunk, lane);
+      flush_unit(cmp, a, s_pfx, b, warp, j_first, j, np, chunk, lane);
       if (r < n - 1) {
-        if (++g == kKvHeads) {
-          g = 0;
-          do {
-            ++b;
-          } while (s_pfx[b + 1] == s_pfx[b]);
-        }
+        do {
+          ++b;
+        } while (s_pfx[b + 1] == s_pfx[b]);
         j = 0;
         j_first = 0;
         np = s_pfx[b + 1] - s_pfx[b];
-        L = s_len[b];
-        cmp.begin(a.q + (static_cast<int64_t>(b) * kQHeads + g * kGroup) * kDim, lane);
+        Lb = s_len[b];
+        need_q = true;
       }
     } else {
       ++j;
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV merge: one CTA per (kv head g, sequence b) unit that decode split
+// into K > 1 pieces.  Warp w merges pieces w, w + 8, ... into a record in
+// shared memory; warp 0 then merges the 8 records (a fixed order) and writes
+// the output rows.  Runs after decode (stream order, or PDL-overlapped
+// launch followed by griddepcontrol.wait).
+// ---------------------------------------------------------------------------
+constexpr int kMergeWarps = 8;
+
+__global__ void __launch_bounds__(kMergeWarps * 32)
+    merge_kernel(const DecodeArgs a, int32_t decode_grid) {
+  __shared__ __align__(16) float s_part[kMergeWarps][kPartialFloats];
+  pdl_wait();
+  pdl_trigger();
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int2 sp = a.meta[b];
+  const int K = sp.y;
+  if (K <= 1) return;
+  const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + sp.x;
+  const int parts = min(kMergeWarps, K);
+  if (warp < parts) {
+    const int cnt = (K - warp + kMergeWarps - 1) / kMergeWarps;
+    merge_partials<false>(a.partials + (S0 + warp) * kPartialFloats, cnt, kMergeWarps,
+                          s_part[warp], false, lane);
+  }
+  __syncthreads();
+  if (warp == 0)
+    merge_partials<true>(&s_part[0][0], parts, 1,
+                         a.out + (static_cast<int64_t>(b) * kQHeads + g * kGroup) * kDim, true,
+                         lane);
 }
 
 // ---------------------------------------------------------------- host side --
@@ -542,15 +880,21 @@ static const void* kernel_ptr() {
 static const void* kernel_for(int kernel) {
   switch (kernel) {
     case PKV_KERNEL_SIMT: return kernel_ptr<SimtCompute>();
+    case PKV_KERNEL_MMA: return kernel_ptr<MmaCompute>();
     default: return nullptr;
   }
+}
+
+static size_t smem_for(int kernel, int32_t batch) {
+  return kernel == PKV_KERNEL_SIMT ? SmemPlan<SimtCompute>::bytes(batch)
+                                   : SmemPlan<MmaCompute>::bytes(batch);
 }
 
 cudaError_t prepare_decode_kernels(int device) {
   int optin = 0;
   cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
   if (e != cudaSuccess) return e;
-  for (int k : {PKV_KERNEL_SIMT}) {
+  for (int k : {PKV_KERNEL_SIMT, PKV_KERNEL_MMA}) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, kernel_for(k));
     if (e != cudaSuccess) return e;
@@ -563,43 +907,66 @@ cudaError_t prepare_decode_kernels(int device) {
 
 int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,
                 DecodePlan* plan) {
-  if (kernel == PKV_KERNEL_AUTO) kernel = PKV_KERNEL_SIMT;
+  if (kernel == PKV_KERNEL_AUTO) kernel = PKV_KERNEL_MMA;
   const void* fn = kernel_for(kernel);
   if (!fn) return PKV_ERR_UNSUPPORTED;
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) !=
       cudaSuccess)
     return PKV_ERR_CUDA;
-  const size_t smem = decode_smem_bytes(batch);
+  const size_t smem = smem_for(kernel, batch);
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return PKV_ERR_CUDA;
   if (smem + fa.sharedSizeBytes > static_cast<size_t>(optin)) return PKV_ERR_UNSUPPORTED;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kWarps * 32, smem) !=
-      cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kWarps * 32, smem) != cudaSuccess)
     return PKV_ERR_CUDA;
   if (per_sm < 1) return PKV_ERR_UNSUPPORTED;
   plan->kernel = kernel;
-  plan->warps = kWarps;
+  plan->threads = kWarps * 32;
   plan->smem = smem;
   plan->grid = grid_ctas > 0 ? grid_ctas : sm_count * per_sm;
-  const int64_t units = static_cast<int64_t>(batch) * kKvHeads;
-  const int64_t W = static_cast<int64_t>(plan->grid) * kWarps;
-  plan->counters_bytes = ((units * 4 + 255) / 256) * 256;
-  plan->ws_bytes = plan->counters_bytes +
-                   static_cast<size_t>(units + W) * kPartialFloats * sizeof(float);
+  const int64_t slots = static_cast<int64_t>(kKvHeads) * (batch + plan->grid);
+  plan->meta_bytes = ((static_cast<int64_t>(batch) * 8 + 255) / 256) * 256;
+  plan->ws_bytes = plan->meta_bytes + static_cast<size_t>(slots) * kPartialFloats * sizeof(float);
   return PKV_OK;
 }
 
+template <class C>
+static cudaError_t launch_one(const DecodePlan& plan, const CUtensorMap& tmap, const DecodeArgs& a,
+                              int flags, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.grid);
+  cfg.blockDim = dim3(plan.threads);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<C>, tmap, a);
+}
+
 cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const DecodeArgs& a,
-                          cudaStream_t stream) {
+                          int flags, cudaStream_t stream) {
+  cudaError_t e;
   switch (plan.kernel) {
-    case PKV_KERNEL_SIMT:
-      decode_kernel<SimtCompute><<<plan.grid, plan.warps * 32, plan.smem, stream>>>(tmap, a);
-      break;
+    case PKV_KERNEL_SIMT: e = launch_one<SimtCompute>(plan, tmap, a, flags, stream); break;
+    case PKV_KERNEL_MMA: e = launch_one<MmaCompute>(plan, tmap, a, flags, stream); break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kKvHeads, a.batch);
+  cfg.blockDim = dim3(kMergeWarps * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, merge_kernel, a, static_cast<int32_t>(plan.grid));
 }
 
 }  // namespace pkv

@@ -14,7 +14,8 @@ struct pkv_pool {
   int device;
   int sm_count;
   int32_t* d_err;
-  CUtensorMap tmap;  // 2-D view of the pool: 64 BF16 x (num_pages * 256) rows
+  int launch_flags;  // PKV_LAUNCH_* bits applied to this pool's kernel launches
+  CUtensorMap tmap;  // 2-D view of the pool: rows of 64 BF16, one 256-row box per page
 };
 
 namespace {
@@ -100,6 +101,7 @@ int pkv_pool_create(int32_t num_pages, int32_t page_tokens, int32_t num_kv_heads
   pkv_pool* p = new (std::nothrow) pkv_pool();
   if (!p) return PKV_ERR_INVALID_ARG;
   p->num_pages = num_pages;
+  p->launch_flags = 0;
   cudaError_t e = cudaGetDevice(&p->device);
   if (e == cudaSuccess)
     e = cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device);
@@ -133,7 +135,7 @@ int pkv_pool_create(int32_t num_pages, int32_t page_tokens, int32_t num_kv_heads
   const cuuint64_t dims[2] = {PKV_HEAD_DIM,
                               static_cast<cuuint64_t>(num_pages) * pkv::kRowsPerPage};
   const cuuint64_t strides[1] = {pkv::kRowBytes};
-  const cuuint32_t box[2] = {PKV_HEAD_DIM, PKV_PAGE_TOKENS};
+  const cuuint32_t box[2] = {PKV_HEAD_DIM, pkv::kRowsPerPage};
   const cuuint32_t elem_strides[2] = {1, 1};
   CUresult r = encode(&p->tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p->data, dims, strides, box,
                       elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -177,8 +179,15 @@ int pkv_append(pkv_pool* pool, const int32_t* block_tables, const int32_t* seq_l
   return from_cuda(pkv::launch_append(
       reinterpret_cast<const __nv_bfloat16*>(k_new), reinterpret_cast<const __nv_bfloat16*>(v_new),
       static_cast<__nv_bfloat16*>(pool->data), layer_slab(block_tables, layer, batch, max_blocks),
-      seq_lens, pool->d_err, batch, max_blocks, pool->num_pages,
+      seq_lens, pool->d_err, batch, max_blocks, pool->num_pages, pool->launch_flags,
       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pkv_pool_set_launch_flags(pkv_pool* pool, int32_t flags) {
+  if (!pool || (flags & ~(PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES))) return PKV_ERR_INVALID_ARG;
+  if ((flags & PKV_LAUNCH_EARLY_TABLES) && !(flags & PKV_LAUNCH_PDL)) return PKV_ERR_INVALID_ARG;
+  pool->launch_flags = flags;
+  return PKV_OK;
 }
 
 int pkv_decode_workspace_bytes_ex(const pkv_pool* pool, int32_t batch, int32_t kernel,
@@ -216,15 +225,18 @@ int paged_attention_decode_ex(const uint16_t* q, const pkv_pool* pool,
   a.bt = layer_slab(block_tables, layer, batch, max_blocks);
   a.seq_lens = seq_lens;
   a.out = out;
-  a.counters = static_cast<int32_t*>(workspace);
-  a.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.counters_bytes);
+  char* ws = static_cast<char*>(workspace);
+  a.meta = reinterpret_cast<int2*>(ws);
+  a.partials = reinterpret_cast<float*>(ws + plan.meta_bytes);
   a.err = pool->d_err;
   a.batch = batch;
   a.max_blocks = max_blocks;
   a.num_pages = pool->num_pages;
   a.min_chunk = min_chunk;
   a.scale_log2 = scale * 1.4426950408889634f;
-  return from_cuda(pkv::launch_decode(plan, pool->tmap, a, reinterpret_cast<cudaStream_t>(stream)));
+  a.flags = pool->launch_flags;
+  return from_cuda(pkv::launch_decode(plan, pool->tmap, a, pool->launch_flags,
+                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int paged_attention_decode(const uint16_t* q, const pkv_pool* pool, const int32_t* block_tables,

@@ -109,6 +109,58 @@ __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap* m
       : "memory");
 }
 
+// 1-D bulk copy (no multicast) of `bytes` (multiple of 16, both addresses
+// 16-byte aligned) from global to shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Four 8x8 b16 matrices from shared memory; lane i gives the address of row
+// i % 8 of matrix i / 8.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// D += A (16x16, row) * B (16x8, col); BF16 inputs, FP32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two floats -> BF16 pair (round to nearest even); `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -130,45 +182,62 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
 
 // ------------------------------------------------------------ launch glue --
 
+// Work-partition cost of one sequence, in pages, on top of its pages (the
+// per-sequence fixed work: query load, softmax finalisation, output).
+constexpr int kSeqCost = 1;
+
+// Launch flags (pool-wide).
+constexpr int kLaunchPdl = 1;         // programmatic dependent launch
+constexpr int kLaunchEarlyTables = 2; // read seq_lens / block tables before waiting
+
 struct DecodeArgs {
   const __nv_bfloat16* q;   // [B][32][64]
   const int32_t* bt;        // this layer's block-table slab [B][max_blocks]
   const int32_t* seq_lens;  // [B]
   float* out;               // [B][32][64]
-  float* partials;          // [8B + W - 1][kPartialFloats]
-  int32_t* counters;        // [8B]
+  float* partials;          // [8 kv heads][B + grid][kPartialFloats]
+  int2* meta;               // [B]: (first CTA, pieces) of each sequence's split
   int32_t* err;             // sticky device error word
   int32_t batch;
   int32_t max_blocks;
   int32_t num_pages;
-  int32_t min_chunk;        // minimum (page, kv head) tiles per warp
+  int32_t min_chunk;        // minimum pages per CTA range
   float scale_log2;         // scale * log2(e)
+  int32_t flags;            // kLaunch* bits
 };
 
 // Launch planning shared by the workspace query and the launch.
 struct DecodePlan {
   int kernel;        // PKV_KERNEL_SIMT or PKV_KERNEL_MMA
   int grid;          // CTAs
-  int warps;         // warps per CTA
+  int threads;       // threads per CTA
   size_t smem;       // dynamic shared memory bytes
   size_t ws_bytes;   // workspace bytes
-  size_t counters_bytes;
+  size_t meta_bytes;
 };
 
 int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,
                 DecodePlan* plan);
 cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const DecodeArgs& a,
-                          cudaStream_t stream);
+                          int flags, cudaStream_t stream);
 cudaError_t prepare_decode_kernels(int device);
 
 cudaError_t launch_append(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
                           __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,
                           int32_t* err, int32_t batch, int32_t max_blocks, int32_t num_pages,
-                          cudaStream_t stream);
+                          int flags, cudaStream_t stream);
 
 cudaError_t launch_gather(const __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,
                           __nv_bfloat16* k_out, __nv_bfloat16* v_out, int32_t* err,
                           int32_t batch, int32_t max_blocks, int32_t num_pages,
                           int32_t max_seq_len, cudaStream_t stream);
+
+// Programmatic dependent launch: wait for the preceding kernel of the stream
+// (no-op when the launch has no programmatic dependency), and allow the next
+// kernel to start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 }  // namespace pkv

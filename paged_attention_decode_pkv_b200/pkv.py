@@ -14,7 +14,7 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpkv.so")
+LIB_PATH = os.environ.get("PKV_LIBRARY") or os.path.join(_HERE, "libpkv.so")
 
 PAGE_TOKENS = 16
 NUM_KV_HEADS = 8
@@ -23,6 +23,8 @@ HEAD_DIM = 64
 PAGE_BYTES = 32768
 
 KERNEL_AUTO, KERNEL_SIMT, KERNEL_MMA = 0, 1, 2
+LAUNCH_PDL = 1
+LAUNCH_EARLY_TABLES = 2
 
 OK = 0
 ERR_INVALID_ARG = -1
@@ -38,7 +40,7 @@ EXPORTS = (
     "pkv_pool_create", "pkv_pool_destroy", "pkv_pool_data", "pkv_pool_num_pages", "pkv_append",
     "pkv_decode_workspace_bytes", "pkv_decode_workspace_bytes_ex", "paged_attention_decode",
     "paged_attention_decode_ex", "pkv_gather", "pkv_get_device_error", "pkv_status_string",
-    "pkv_last_error_message",
+    "pkv_last_error_message", "pkv_pool_set_launch_flags",
 )
 
 
@@ -64,6 +66,7 @@ def _load():
         "pkv_get_device_error": ([P, P, ctypes.POINTER(i32)], ctypes.c_int),
         "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "pkv_last_error_message": ([], ctypes.c_char_p),
+        "pkv_pool_set_launch_flags": ([P, i32], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -155,6 +158,10 @@ class Pool:
         except Exception:
             pass
 
+    def set_launch_flags(self, flags: int):
+        """PKV_LAUNCH_* bits for this pool's later kernel launches."""
+        _check(lib.pkv_pool_set_launch_flags(self.handle, int(flags)), "pkv_pool_set_launch_flags")
+
     def workspace_bytes(self, batch: int, kernel: int = KERNEL_AUTO, grid_ctas: int = 0) -> int:
         n = ctypes.c_size_t()
         with torch.cuda.device(self.device):
@@ -164,11 +171,11 @@ class Pool:
         return n.value
 
     def workspace(self, batch: int, kernel: int = KERNEL_AUTO, grid_ctas: int = 0) -> torch.Tensor:
-        """A zero-initialised workspace, cached per (batch, kernel, grid)."""
+        """A decode workspace, cached per (batch, kernel, grid)."""
         key = (int(batch), int(kernel), int(grid_ctas))
         ws = self._ws.get(key)
         if ws is None:
-            ws = torch.zeros(max(256, self.workspace_bytes(*key)), dtype=torch.uint8,
+            ws = torch.empty(max(256, self.workspace_bytes(*key)), dtype=torch.uint8,
                              device=self.device)
             self._ws[key] = ws
         return ws

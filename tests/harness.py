@@ -13,7 +13,7 @@ from paged_attention_decode_pkv_b200 import pkv
 from paged_attention_decode_pkv_b200 import workloads as W
 
 ATOL = 2e-3
-KERNELS = [pkv.KERNEL_SIMT]
+KERNELS = [pkv.KERNEL_SIMT, pkv.KERNEL_MMA]
 
 
 def bits(t):

@@ -34,7 +34,7 @@ def test_decode_edge_lengths(kernel, lens):
 
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("grid,min_chunk", [(1, 0), (2, 0), (7, 0), (3, 1), (0, 1), (0, 3),
-                                            (0, 64), (50, 2)])
+                                            (0, 64), (50, 2), (100, 1), (77, 0)])
 def test_decode_split_patterns(kernel, grid, min_chunk):
     # Different grids / chunk sizes cut the (sequence, kv head) runs at
     # different places, exercising the split-KV merge; the result must stay
@@ -159,3 +159,27 @@ def test_scale_and_layer_arguments():
         for scale in (0.0, 0.125, 0.5):
             got = g.decode(layer=layer, scale=scale)
             assert max_err(got, g.oracle(layer=layer, scale=scale)) <= ATOL
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_programmatic_dependent_launch_keeps_results(kernel):
+    # With PDL each kernel waits for its predecessor before touching memory,
+    # so an append followed by decodes must give the same answer.
+    c = make_case([40, 1, 77, 16], seed=31, spare_pages=3)
+    g = GpuCase(c)
+    g.pool.set_launch_flags(pkv.LAUNCH_PDL)
+    pkv.append(g.pool, g.bt, g.sl, u16_to_bf16(c["k_new"]), u16_to_bf16(c["v_new"]), 0)
+    first = g.decode(kernel=kernel)
+    for _ in range(5):
+        pkv.append(g.pool, g.bt, g.sl, u16_to_bf16(c["k_new"]), u16_to_bf16(c["v_new"]), 0)
+        assert np.array_equal(g.decode(kernel=kernel), first)
+    assert max_err(first, g.oracle()) <= ATOL
+    assert pkv.get_device_error(g.pool) == 0
+    with pytest.raises(pkv.PkvError):
+        g.pool.set_launch_flags(4)
+    with pytest.raises(pkv.PkvError):
+        g.pool.set_launch_flags(pkv.LAUNCH_EARLY_TABLES)   # needs PDL
+    g.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES)
+    for _ in range(3):
+        pkv.append(g.pool, g.bt, g.sl, u16_to_bf16(c["k_new"]), u16_to_bf16(c["v_new"]), 0)
+        assert np.array_equal(g.decode(kernel=kernel), first)
