@@ -85,7 +85,8 @@ typedef enum {
   PKV_ERR_BAD_PAGE = -5,       /* device: block-table entry outside [0, num_pages)  */
   PKV_ERR_WORKSPACE = -6,      /* workspace missing, misaligned or too small        */
   PKV_ERR_DEVICE_TIMEOUT = -7, /* device: a bounded wait on a copy ran out           */
-  PKV_ERR_BAD_SEQ_LEN = -8     /* device: seq_len < 0 (append: < 1) or too long      */
+  PKV_ERR_BAD_SEQ_LEN = -8,    /* device: seq_len < 0 (append: < 1) or too long      */
+  PKV_ERR_TOO_LARGE = -9       /* batch too large for the fixed no-alloc scratch     */
 } pkv_status;
 
 /* Launch flags for pkv_pool_set_launch_flags. */
@@ -212,6 +213,34 @@ PKV_API int pkv_decode_workspace_bytes_ex(const pkv_pool *pool, int32_t batch, i
 PKV_API int pkv_gather(const pkv_pool *pool, const int32_t *block_tables, const int32_t *seq_lens,
                int32_t layer, uint16_t *k_out, uint16_t *v_out, int32_t num_layers,
                int32_t batch, int32_t max_blocks, int32_t max_seq_len, pkv_stream_t stream);
+
+/*
+ * Allocation-free decode (the pages have no counterpart: this entry point
+ * exists for callers that cannot allocate device memory where they run
+ * attention -- code running inside an allocator or memory-pool callback,
+ * runtime plugins that receive only their inputs and outputs, or loops that
+ * must never call cudaMalloc/cudaFree because those calls synchronise the
+ * device).  Same computation, arguments and device-error behaviour as
+ * paged_attention_decode, but instead of a caller workspace it uses a
+ * scratch area of PKV_NOALLOC_SCRATCH_BYTES that the library keeps in every
+ * GPU's memory from load until process exit.  It allocates nothing.
+ *  - Limit: returns PKV_ERR_TOO_LARGE (nothing launched) when the batch
+ *    needs more scratch than that (pkv_decode_workspace_bytes > limit); on a
+ *    B200 with the default grid this allows about 1,600 sequences.
+ *  - The first call on a device looks up the scratch's device address
+ *    (cudaGetSymbolAddress, with the pool's device current); make that first
+ *    call before any stream capture.
+ *  - All calls on one device share the one scratch area, which keeps the
+ *    last call's contents; nothing in it has to start at zero.  Calls whose
+ *    kernels overlap on the GPU (different streams, or different threads
+ *    without ordering) race on it and give wrong results: serialise them.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+PKV_API int paged_attention_decode_noalloc(const uint16_t *q, const pkv_pool *pool,
+                                           const int32_t *block_tables, const int32_t *seq_lens,
+                                           int32_t layer, float scale, float *out,
+                                           int32_t num_layers, int32_t batch, int32_t max_blocks,
+                                           pkv_stream_t stream);
 
 /* Synchronise `stream`, return in *status_out the first device error
  * recorded since the last call (PKV_OK if none) and clear it. */

@@ -3,6 +3,7 @@
 // Host-visible argument errors are caught here before anything is launched;
 // everything else is the kernels' business (see pkv.h for the contract).
 #include <cstdio>
+#include <mutex>
 #include <new>
 
 #include "pkv_internal.cuh"
@@ -279,6 +280,71 @@ int pkv_get_device_error(pkv_pool* pool, pkv_stream_t stream, int32_t* status_ou
   return PKV_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free decode.
+//
+// Some callers cannot allocate device memory at the point where they run
+// attention: code that executes inside a custom memory-pool or allocator
+// callback (where re-entering the allocator deadlocks or corrupts its
+// state), plugins for inference runtimes that hand a kernel only its
+// inputs and outputs, or real-time loops that must never call
+// cudaMalloc/cudaFree because those calls synchronise the device.  For them
+// paged_attention_decode_noalloc uses a fixed scratch area that the library
+// reserves in device memory when it is loaded, instead of a caller-provided
+// workspace.  The area is a file-scope __device__ array (so every GPU that
+// loads the library holds it until the process exits); its size bounds the
+// batch (pkv.h gives the limit).  The host needs the array's device address,
+// which is not the host-side symbol: it is looked up once per device with
+// cudaGetSymbolAddress, with that device current, on the first call.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[256];   // per device ordinal; nullptr until looked up
+
+// Device address of this device's scratch array (looked up on first use).
+int scratch_for_device(int device, void** out) {
+  if (device < 0 || device >= 256) return PKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[device]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return from_cuda(e == cudaSuccess ? cudaErrorInvalidSymbol : e,
+                                                 "paged_attention_decode_noalloc: scratch address");
+    g_scratch_addr[device] = p;
+  }
+  *out = g_scratch_addr[device];
+  return PKV_OK;
+}
+}  // namespace
+
+int paged_attention_decode_noalloc(const uint16_t* q, const pkv_pool* pool,
+                                   const int32_t* block_tables, const int32_t* seq_lens,
+                                   int32_t layer, float scale, float* out, int32_t num_layers,
+                                   int32_t batch, int32_t max_blocks, pkv_stream_t stream) {
+  int s = check_table_args(pool, block_tables, seq_lens, layer, num_layers, batch, max_blocks);
+  if (s != PKV_OK) return s;
+  size_t need = 0;
+  s = pkv_decode_workspace_bytes(pool, batch, &need);
+  if (s != PKV_OK) return s;
+  if (need > sizeof(g_noalloc_scratch)) {
+    snprintf(g_last_error, sizeof g_last_error,
+             "paged_attention_decode_noalloc: batch %d needs %zu scratch bytes, the fixed scratch "
+             "holds %zu",
+             batch, need, sizeof(g_noalloc_scratch));
+    return PKV_ERR_TOO_LARGE;
+  }
+  void* scratch = nullptr;
+  s = scratch_for_device(pool->device, &scratch);
+  if (s != PKV_OK) return s;
+  // Nothing in the workspace has to start at zero (each decode writes the
+  // split table and the partial records before reading them), so the shared
+  // scratch needs no clearing between calls.
+  return paged_attention_decode(q, pool, block_tables, seq_lens, layer, scale, out, num_layers,
+                                batch, max_blocks, scratch, sizeof(g_noalloc_scratch), stream);
+}
+
 const char* pkv_last_error_message(void) { return g_last_error; }
 
 const char* pkv_status_string(int status) {
@@ -292,6 +358,7 @@ const char* pkv_status_string(int status) {
     case PKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case PKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case PKV_ERR_BAD_SEQ_LEN: return "sequence length out of range";
+    case PKV_ERR_TOO_LARGE: return "request larger than the fixed no-alloc scratch";
     default: return "unknown status";
   }
 }

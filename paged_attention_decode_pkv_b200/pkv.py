@@ -35,12 +35,14 @@ ERR_BAD_PAGE = -5
 ERR_WORKSPACE = -6
 ERR_DEVICE_TIMEOUT = -7
 ERR_BAD_SEQ_LEN = -8
+ERR_TOO_LARGE = -9
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTS = (
     "pkv_pool_create", "pkv_pool_destroy", "pkv_pool_data", "pkv_pool_num_pages", "pkv_append",
     "pkv_decode_workspace_bytes", "pkv_decode_workspace_bytes_ex", "paged_attention_decode",
     "paged_attention_decode_ex", "pkv_gather", "pkv_get_device_error", "pkv_status_string",
-    "pkv_last_error_message", "pkv_pool_set_launch_flags",
+    "pkv_last_error_message", "pkv_pool_set_launch_flags", "paged_attention_decode_noalloc",
 )
 
 
@@ -67,6 +69,8 @@ def _load():
         "pkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "pkv_last_error_message": ([], ctypes.c_char_p),
         "pkv_pool_set_launch_flags": ([P, i32], ctypes.c_int),
+        "paged_attention_decode_noalloc": ([P, P, P, P, i32, ctypes.c_float, P, i32, i32, i32, P],
+                                           ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -207,6 +211,24 @@ def decode(q: torch.Tensor, pool: Pool, block_tables: torch.Tensor, seq_lens: to
         _dev(out, torch.float32, (B, NUM_Q_HEADS, HEAD_DIM), "out"), L, B, MB,
         _dev(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream),
         int(kernel), int(grid_ctas), int(min_chunk)), "paged_attention_decode")
+    return out
+
+
+def decode_noalloc(q: torch.Tensor, pool: Pool, block_tables: torch.Tensor,
+                   seq_lens: torch.Tensor, layer: int, scale: float, out: torch.Tensor,
+                   stream=None) -> torch.Tensor:
+    """Decode through paged_attention_decode_noalloc: no workspace argument,
+    nothing allocated by the library (it uses its own fixed device scratch).
+    For callers that cannot allocate device memory where attention runs;
+    `out` must therefore be passed in.  Calls that overlap on the GPU share
+    the scratch and race."""
+    L, B, MB = block_tables.shape
+    _check(lib.paged_attention_decode_noalloc(
+        _dev(q, torch.bfloat16, (B, NUM_Q_HEADS, HEAD_DIM), "q"), pool.handle,
+        _dev(block_tables, torch.int32, None, "block_tables"),
+        _dev(seq_lens, torch.int32, (B,), "seq_lens"), int(layer), float(scale),
+        _dev(out, torch.float32, (B, NUM_Q_HEADS, HEAD_DIM), "out"), L, B, MB, _stream(stream)),
+        "paged_attention_decode_noalloc")
     return out
 
 
