@@ -116,6 +116,40 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------- multi-rank --
+# The path shards by sequence with no exchange: each rank runs its own
+# replica of the workload (its own pool, block tables and sequences, seeded
+# per rank), so per-GPU work is fixed as ranks are added (weak scaling) and
+# the only collectives are the barrier around the timed region and the max
+# of the elapsed times.
+
+def workload_for_rank(name: str, rank: int) -> W.Workload:
+    """Rank r gets the same workload shape drawn with seed + 1000 r."""
+    base = W.make(name)
+    return base if rank == 0 else W.make(name, seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Largest `value` over all ranks (identity without a process group)."""
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as tdist
+    if tdist.is_available() and tdist.is_initialized():
+        tdist.barrier()
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Units processed by all ranks per second of the slowest rank."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 # ---------------------------------------------------------------- our arm --
 
 class Runner:
@@ -187,21 +221,12 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     kernel = {"auto": pkv.KERNEL_AUTO, "simt": pkv.KERNEL_SIMT, "mma": pkv.KERNEL_MMA}[args.kernel]
-    w = W.make(args.workload, seed=W.make(args.workload).seed + 1000 * rank) if rank else \
-        W.make(args.workload)
+    w = workload_for_rank(args.workload, rank)
     r = Runner(w, device, kernel)
     if not args.no_pdl:
         # appends precede every decode and only read the tables
         r.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES)
     stream = torch.cuda.Stream(device)
-    dist = world > 1
-    if dist:
-        import torch.distributed as tdist
-
-    def barrier():
-        if dist:
-            tdist.barrier()
-
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             r.launch_step(stream, i % w.num_steps)
@@ -232,15 +257,11 @@ def run_ours(args, rank, world, local_rank):
     err = pkv.get_device_error(r.pool, stream)
     if err != 0:
         raise RuntimeError("device error during timed region: %s" % pkv.status_string(err))
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
-    queries = args.steps * w.num_layers * w.batch * world
-    value = queries / (ms / 1e3)
+    ms = max_over_ranks(ms, device)
+    value = whole_job_rate(args.steps * w.num_layers * w.batch, world, ms)
 
     # ---- end to end through the public API from pinned host buffers
-    e2e = run_e2e(r, stream, min(args.steps, args.e2e_steps), barrier, dist, device)
+    e2e = run_e2e(r, stream, min(args.steps, args.e2e_steps), device, world)
 
     if rank != 0:
         return None
@@ -281,7 +302,7 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
-def run_e2e(r: Runner, stream, steps, barrier, dist, device):
+def run_e2e(r: Runner, stream, steps, device, world):
     """Same step through the public API, with every step's inputs (q, k_new,
     v_new of all layers, seq_lens) copied from pinned host memory before the
     step's graph runs and all outputs copied back to pinned host memory."""
@@ -309,21 +330,10 @@ def run_e2e(r: Runner, stream, steps, barrier, dist, device):
         t1.record(stream)
     stream.synchronize()
     barrier()
-    ms = t0.elapsed_time(t1)
-    if dist:
-        import torch.distributed as tdist
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
-    world = tdist_world() if dist else 1
-    return {"value": steps * w.num_layers * w.batch * world / (ms / 1e3), "unit": UNIT,
+    ms = max_over_ranks(t0.elapsed_time(t1), device)
+    return {"value": whole_job_rate(steps * w.num_layers * w.batch, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps}
-
-
-def tdist_world():
-    import torch.distributed as tdist
-    return tdist.get_world_size()
 
 
 # ------------------------------------------------------------ oracle arms --

@@ -93,6 +93,9 @@ typedef enum {
 #define PKV_LAUNCH_PDL 1          /* programmatic dependent launch (see below) */
 #define PKV_LAUNCH_EARLY_TABLES 2 /* with PDL: decode reads seq_lens and block
                                      tables before the preceding kernel ends */
+#define PKV_LAUNCH_TEST_STALL (1 << 30) /* testing only: decode withholds one
+                                     page so its bounded waits run out (~1 s)
+                                     and it reports PKV_ERR_DEVICE_TIMEOUT */
 
 /* Decode kernel variants for paged_attention_decode_ex. */
 #define PKV_KERNEL_AUTO 0
@@ -136,8 +139,13 @@ PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
  * overlaps that kernel; the caller guarantees that the kernel launched just
  * before a decode does not write seq_lens or the block tables (an append,
  * which only reads them, is fine).
- * flags: 0, PKV_LAUNCH_PDL or PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES, else
- * PKV_ERR_INVALID_ARG.
+ * PKV_LAUNCH_TEST_STALL exists only to test the device-timeout path: the
+ * decode kernel never fills one shared-memory stage, every wait on it gives
+ * up after about a second, the kernel exits early with garbage output and
+ * pkv_get_device_error reports PKV_ERR_DEVICE_TIMEOUT; the context stays
+ * usable.
+ * flags: 0, PKV_LAUNCH_PDL or PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES,
+ * optionally | PKV_LAUNCH_TEST_STALL, else PKV_ERR_INVALID_ARG.
  */
 PKV_API int pkv_pool_set_launch_flags(pkv_pool *pool, int32_t flags);
 

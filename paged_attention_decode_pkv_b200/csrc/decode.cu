@@ -741,7 +741,12 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   }
   if (n <= 0) return;
   // Issue page r into stage r % kS (warp 0 only; stage known to be free).
+  // Test-only: leave page 0's full barrier unarmed, so the consumers' bounded
+  // waits run out and the launch reports PKV_ERR_DEVICE_TIMEOUT.
+  const bool stall = (a.flags & kLaunchTestStall) != 0;
+  int issued = 0;   // pages issued so far (warp 0)
   auto issue = [&](int r) {
+    ++issued;
     if ((r >> 5) != cur_k) {
       cur_phys = nxt_phys;
       cur_info = nxt_info;
@@ -750,7 +755,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
     }
     const int32_t phys = __shfl_sync(kFull, cur_phys, r & 31);
     const int32_t info = __shfl_sync(kFull, cur_info, r & 31);
-    if (lane == 0) {
+    if (lane == 0 && !(stall && r == 0)) {
       const int st = r % kS;
       const uint32_t bar = full + 8 * st;
       const uint32_t dst = base + L::stages + st * kStageBytes;
@@ -772,6 +777,14 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   };
   if (warp == 0)
     for (int r = 0; r < n && r < kS; ++r) issue(r);
+  // After a timed-out wait: wait (bounded) for the copies still in flight
+  // into this CTA's stages, pages k0 .. issued-1, before the CTA exits.
+  auto drain = [&](int k0) {
+    if (warp != 0) return;
+    for (int k = k0; k < issued; ++k)
+      if (!(stall && k == 0))
+        mbar_wait_bounded(full + 8 * (k % kS), static_cast<uint32_t>(k / kS) & 1u);
+  };
 
   // ---- consumers (all 8 warps; warp g computes kv head g)
   int b, j;
@@ -792,9 +805,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
       if (!mbar_try_wait(eb, par) && !mbar_wait_bounded(eb, par)) {
         if (lane == 0) record_error(a.err, kErrTimeout);
         s_flags[kS] = 1;
-        // copies already issued land in stages r-1+1 .. r-2+kS; wait for them
-        for (int k = r; k < r - 1 + kS && k < n; ++k)
-          mbar_wait_bounded(full + 8 * (k % kS), static_cast<uint32_t>(k / kS) & 1u);
+        drain(r);
         return;
       }
       issue(rr + kS);
@@ -804,9 +815,13 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
     if (!mbar_try_wait(fb, par) && !mbar_wait_bounded(fb, par)) {
       if (lane == 0) record_error(a.err, kErrTimeout);
       s_flags[kS] = 1;
+      drain(r + 1);
       return;
     }
-    if (s_flags[kS]) return;   // another warp gave up; results are void
+    if (s_flags[kS]) {   // another warp gave up; results are void
+      drain(r + 1);
+      return;
+    }
     const uint32_t stage = base + L::stages + st * kStageBytes;
     if (need_q) {
       cmp.begin(stage + kPageBytes + warp * (kGroup * kRowBytes), lane);

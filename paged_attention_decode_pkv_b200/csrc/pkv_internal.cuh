@@ -189,6 +189,7 @@ constexpr int kSeqCost = 1;
 // Launch flags (pool-wide).
 constexpr int kLaunchPdl = 1;         // programmatic dependent launch
 constexpr int kLaunchEarlyTables = 2; // read seq_lens / block tables before waiting
+constexpr int kLaunchTestStall = PKV_LAUNCH_TEST_STALL;  // testing the timeout path only
 
 struct DecodeArgs {
   const __nv_bfloat16* q;   // [B][32][64]

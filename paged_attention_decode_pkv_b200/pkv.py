@@ -25,6 +25,7 @@ PAGE_BYTES = 32768
 KERNEL_AUTO, KERNEL_SIMT, KERNEL_MMA = 0, 1, 2
 LAUNCH_PDL = 1
 LAUNCH_EARLY_TABLES = 2
+LAUNCH_TEST_STALL = 1 << 30
 
 OK = 0
 ERR_INVALID_ARG = -1

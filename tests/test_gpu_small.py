@@ -183,3 +183,18 @@ def test_programmatic_dependent_launch_keeps_results(kernel):
     for _ in range(3):
         pkv.append(g.pool, g.bt, g.sl, u16_to_bf16(c["k_new"]), u16_to_bf16(c["v_new"]), 0)
         assert np.array_equal(g.decode(kernel=kernel), first)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_bounded_wait_reports_timeout_and_context_survives(kernel):
+    # A stage that nothing fills: every wait on it gives up after ~1 s, the
+    # kernel reports PKV_ERR_DEVICE_TIMEOUT, and the next launch works.
+    c = make_case([40, 300, 17], seed=37, spare_pages=2)
+    g = GpuCase(c)
+    g.pool.set_launch_flags(pkv.LAUNCH_TEST_STALL)
+    g.decode(kernel=kernel)
+    assert pkv.get_device_error(g.pool) == pkv.ERR_DEVICE_TIMEOUT
+    g.pool.set_launch_flags(0)
+    got = g.decode(kernel=kernel)
+    assert pkv.get_device_error(g.pool) == 0
+    assert max_err(got, g.oracle()) <= ATOL
