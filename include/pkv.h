@@ -165,10 +165,10 @@ PKV_API int pkv_append(pkv_pool *pool, const int32_t *block_tables, const int32_
 /*
  * Workspace bytes paged_attention_decode needs for this batch on the pool's
  * device: the split-KV partial results (m, l and the unnormalised output of
- * every piece of a split sequence) and the per-sequence split table.  The
- * workspace is caller-owned device memory, 256-byte aligned; its contents
- * need no initialisation (every decode writes what it later reads).  Calls
- * that share one workspace must not overlap in time.
+ * every piece of a split sequence).  The workspace is caller-owned device
+ * memory, 256-byte aligned; its contents need no initialisation (every
+ * decode writes what it later reads).  Calls that share one workspace must
+ * not overlap in time.
  */
 PKV_API int pkv_decode_workspace_bytes(const pkv_pool *pool, int32_t batch, size_t *bytes_out);
 

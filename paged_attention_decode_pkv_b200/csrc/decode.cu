@@ -547,6 +547,15 @@ __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stri
   }
   for (int s0 = 0; s0 < cnt; s0 += 32) {
     const int n = min(32, cnt - s0);
+    const float* base = P + s0 * step + 2 * kGroup;
+    // accumulator loads of the first kMergeBatch pieces go out with the m/l loads
+    float2 v[kMergeBatch][kGroup];
+#pragma unroll
+    for (int kk = 0; kk < kMergeBatch; ++kk)
+#pragma unroll
+      for (int h = 0; h < kGroup; ++h)
+        v[kk][h] = (kk < n) ? ld2<kShared>(base + kk * step + h * kDim + 2 * lane)
+                            : make_float2(0.f, 0.f);
     float mm[kGroup] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     float ll[kGroup] = {0.f, 0.f, 0.f, 0.f};
     if (lane < n) {
@@ -573,15 +582,15 @@ __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stri
       wgt[h] = (mm[h] == -INFINITY) ? 0.f : fast_exp2(mm[h] - mn);
       S[h] = fmaf(wgt[h], ll[h], S[h]);
     }
-    const float* base = P + s0 * step + 2 * kGroup;
     for (int k0 = 0; k0 < n; k0 += kMergeBatch) {
-      float2 v[kMergeBatch][kGroup];
+      if (k0 > 0) {
 #pragma unroll
-      for (int kk = 0; kk < kMergeBatch; ++kk)
+        for (int kk = 0; kk < kMergeBatch; ++kk)
 #pragma unroll
-        for (int h = 0; h < kGroup; ++h)
-          v[kk][h] = (k0 + kk < n) ? ld2<kShared>(base + (k0 + kk) * step + h * kDim + 2 * lane)
-                                   : make_float2(0.f, 0.f);
+          for (int h = 0; h < kGroup; ++h)
+            v[kk][h] = (k0 + kk < n) ? ld2<kShared>(base + (k0 + kk) * step + h * kDim + 2 * lane)
+                                     : make_float2(0.f, 0.f);
+      }
 #pragma unroll
       for (int kk = 0; kk < kMergeBatch; ++kk)
 #pragma unroll
@@ -619,12 +628,21 @@ __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stri
 // consecutive slots S0 .. S0 + K - 1 with S0 = g * (B + grid) + b + c_first
 // (b + cta is distinct for every piece of head g because both only grow
 // along the page order).
-__device__ __forceinline__ int2 split_of(const int32_t* s_pfx, int b, int64_t chunk) {
-  const int np = s_pfx[b + 1] - s_pfx[b];
+__device__ __forceinline__ int2 split_of(int64_t pages_before, int b, int np, int64_t chunk) {
   if (np == 0) return make_int2(0, 0);
-  const int64_t first = seq_cost(s_pfx, b) + kSeqCost;
+  const int64_t first = pages_before + static_cast<int64_t>(kSeqCost) * b + kSeqCost;
   const int c_first = static_cast<int>(first / chunk);
   return make_int2(c_first, static_cast<int>((first + np - 1) / chunk) - c_first + 1);
+}
+
+// Pages per CTA range: every sequence costs its pages plus kSeqCost, the
+// total is cut into `grid` equal ranges (at least min_chunk pages).
+__device__ __forceinline__ int64_t range_chunk(int64_t total_pages, int batch, int grid,
+                                               int min_chunk) {
+  const int64_t total = total_pages + static_cast<int64_t>(kSeqCost) * batch;
+  int64_t chunk = (total + grid - 1) / grid;
+  if (chunk < min_chunk) chunk = min_chunk;
+  return chunk < 1 ? 1 : chunk;
 }
 
 // End of a sequence's piece inside this CTA's range, for kv head g (= this
@@ -638,10 +656,8 @@ __device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a,
     cmp.finalize(a.out + (static_cast<int64_t>(b) * kQHeads + g * kGroup) * kDim, lane);
     return;
   }
-  const int2 sp = split_of(s_pfx, b, chunk);
   const int64_t slot = static_cast<int64_t>(g) * (a.batch + gridDim.x) + b + blockIdx.x;
   cmp.store_partial(a.partials + slot * kPartialFloats, lane);
-  (void)sp;
 }
 
 // Producer-side description of page f (this lane's slot of a 32-page batch):
@@ -713,9 +729,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
 
   const int G = gridDim.x;
   const int64_t total = seq_cost(s_pfx, B);
-  int64_t chunk = (total + G - 1) / G;
-  if (chunk < a.min_chunk) chunk = a.min_chunk;
-  if (chunk < 1) chunk = 1;
+  const int64_t chunk = range_chunk(s_pfx[B], B, G, a.min_chunk);
   const int64_t x0 = static_cast<int64_t>(blockIdx.x) * chunk;
   const int32_t p0 = x0 < total ? pages_below(s_pfx, B, x0) : 0;
   const int32_t p1 = x0 < total ? pages_below(s_pfx, B, x0 + chunk) : 0;
@@ -732,13 +746,9 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   }
   if (early) pdl_wait();
 
-  // every sequence once across the grid: its split for the merge kernel, and
-  // zero output rows if it is empty
-  for (int b = blockIdx.x * kWarps + warp; b < B; b += G * kWarps) {
-    const int2 sp = split_of(s_pfx, b, chunk);
-    if (lane == 0) a.meta[b] = sp;
-    if (sp.y == 0) zero_rows(a.out + static_cast<int64_t>(b) * kQHeads * kDim, lane);
-  }
+  // empty (or invalid) sequences: zero output rows, once across the grid
+  for (int b = blockIdx.x * kWarps + warp; b < B; b += G * kWarps)
+    if (s_pfx[b + 1] == s_pfx[b]) zero_rows(a.out + static_cast<int64_t>(b) * kQHeads * kDim, lane);
   if (n <= 0) return;
   // Issue page r into stage r % kS (warp 0 only; stage known to be free).
   // Test-only: leave page 0's full barrier unarmed, so the consumers' bounded
@@ -854,23 +864,54 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
 
 // ---------------------------------------------------------------------------
 // Split-KV merge: one CTA per (kv head g, sequence b) unit that decode split
-// into K > 1 pieces.  Warp w merges pieces w, w + 8, ... into a record in
-// shared memory; warp 0 then merges the 8 records (a fixed order) and writes
-// the output rows.  Runs after decode (stream order, or PDL-overlapped
-// launch followed by griddepcontrol.wait).
+// into K > 1 pieces.  The split is recomputed here from the lengths (an
+// input that nothing in the launch writes), before waiting for the decode
+// grid, so that with programmatic dependent launch only the partial records
+// are read after decode ends.  Warp w merges pieces w, w + 8, ... into a
+// record in shared memory; warp 0 then merges the 8 records (a fixed order)
+// and writes the output rows.
 // ---------------------------------------------------------------------------
 constexpr int kMergeWarps = 8;
 
 __global__ void __launch_bounds__(kMergeWarps * 32)
     merge_kernel(const DecodeArgs a, int32_t decode_grid) {
   __shared__ __align__(16) float s_part[kMergeWarps][kPartialFloats];
-  pdl_wait();
+  __shared__ int32_t s_sum[2][kMergeWarps];
   pdl_trigger();
   const int g = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int2 sp = a.meta[b];
+  const int64_t cap = static_cast<int64_t>(a.max_blocks) * kTokens;
+  int before = 0, all = 0;
+  for (int i = threadIdx.x; i < a.batch; i += blockDim.x) {
+    int L = a.seq_lens[i];
+    if (L < 0 || L > cap) L = 0;
+    const int np = (L + kTokens - 1) / kTokens;
+    all += np;
+    before += (i < b) ? np : 0;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    before += __shfl_xor_sync(kFull, before, off);
+    all += __shfl_xor_sync(kFull, all, off);
+  }
+  if (lane == 0) {
+    s_sum[0][warp] = before;
+    s_sum[1][warp] = all;
+  }
+  __syncthreads();
+  int64_t pages_before = 0, pages_all = 0;
+#pragma unroll
+  for (int k = 0; k < kMergeWarps; ++k) {
+    pages_before += s_sum[0][k];
+    pages_all += s_sum[1][k];
+  }
+  int Lb = a.seq_lens[b];
+  if (Lb < 0 || Lb > cap) Lb = 0;
+  const int64_t chunk = range_chunk(pages_all, a.batch, decode_grid, a.min_chunk);
+  const int2 sp = split_of(pages_before, b, (Lb + kTokens - 1) / kTokens, chunk);
   const int K = sp.y;
   if (K <= 1) return;
+  pdl_wait();   // the pieces are written by the decode grid
   const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + sp.x;
   const int parts = min(kMergeWarps, K);
   if (warp < parts) {
@@ -942,8 +983,7 @@ int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ct
   plan->smem = smem;
   plan->grid = grid_ctas > 0 ? grid_ctas : sm_count * per_sm;
   const int64_t slots = static_cast<int64_t>(kKvHeads) * (batch + plan->grid);
-  plan->meta_bytes = ((static_cast<int64_t>(batch) * 8 + 255) / 256) * 256;
-  plan->ws_bytes = plan->meta_bytes + static_cast<size_t>(slots) * kPartialFloats * sizeof(float);
+  plan->ws_bytes = static_cast<size_t>(slots) * kPartialFloats * sizeof(float);
   return PKV_OK;
 }
 

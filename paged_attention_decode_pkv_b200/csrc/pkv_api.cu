@@ -227,9 +227,7 @@ int paged_attention_decode_ex(const uint16_t* q, const pkv_pool* pool,
   a.bt = layer_slab(block_tables, layer, batch, max_blocks);
   a.seq_lens = seq_lens;
   a.out = out;
-  char* ws = static_cast<char*>(workspace);
-  a.meta = reinterpret_cast<int2*>(ws);
-  a.partials = reinterpret_cast<float*>(ws + plan.meta_bytes);
+  a.partials = static_cast<float*>(workspace);
   a.err = pool->d_err;
   a.batch = batch;
   a.max_blocks = max_blocks;

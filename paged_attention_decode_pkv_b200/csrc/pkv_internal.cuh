@@ -197,7 +197,6 @@ struct DecodeArgs {
   const int32_t* seq_lens;  // [B]
   float* out;               // [B][32][64]
   float* partials;          // [8 kv heads][B + grid][kPartialFloats]
-  int2* meta;               // [B]: (first CTA, pieces) of each sequence's split
   int32_t* err;             // sticky device error word
   int32_t batch;
   int32_t max_blocks;
@@ -214,7 +213,6 @@ struct DecodePlan {
   int threads;       // threads per CTA
   size_t smem;       // dynamic shared memory bytes
   size_t ws_bytes;   // workspace bytes
-  size_t meta_bytes;
 };
 
 int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,
