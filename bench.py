@@ -51,6 +51,36 @@ def alg_bytes_decode(seq_lens: np.ndarray) -> int:
     return int((2048 * L + 4096 + 8192 + 4 * ((L + 15) // 16) + 4).sum())
 
 
+def kernel_source_digest() -> str:
+    """sha256 of the decode kernel's sources (the ncu traffic figure is only
+    valid for the sources it was captured on)."""
+    import hashlib
+    h = hashlib.sha256()
+    for fn in ("decode.cu", "pkv_internal.cuh"):
+        with open(os.path.join(ROOT, "paged_attention_decode_pkv_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str, alg_bytes: float):
+    """DRAM bytes per decode launch from the committed ncu summary of this
+    workload, scaled to `alg_bytes`; None if there is none or the kernel
+    sources changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic_%s.txt" % workload)
+    try:
+        kv = {}
+        with open(p) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel_source_sha256") != kernel_source_digest():
+            return None
+        return float(kv["dram_bytes_per_launch"]) * alg_bytes / float(kv["alg_bytes_of_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -175,45 +205,39 @@ class Runner:
         self.out = torch.empty((nl, B, 32, 64), dtype=torch.float32, device=device)
         self.ws = self.pool.workspace(B, kernel)
 
-    def launch_step(self, stream, variant, events=None, seq_lens=None):
-        """Launch one decode step (all layers) for lengths variant `variant`;
-        optionally record (start, end) events around every decode launch."""
+    def launch_step(self, stream, variant, decode_only=False):
+        """Launch one decode step (all layers) for lengths variant `variant`:
+        append + decode per layer, or only the decodes."""
         pkv = self.pkv
-        sl = self.seq_lens[variant] if seq_lens is None else seq_lens
+        sl = self.seq_lens[variant]
         for l in range(self.w.num_layers):
-            pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
-            if events is not None:
-                events[l][0].record(stream)
+            if not decode_only:
+                pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
             pkv.decode(self.q[l], self.pool, self.bt, sl, l, self.w.scale, out=self.out[l],
                        workspace=self.ws, kernel=self.kernel, stream=stream)
-            if events is not None:
-                events[l][1].record(stream)
 
     def capture(self, stream):
-        """One CUDA graph per lengths variant (the workload's step cycle),
-        each with timing events around its decode launches."""
-        self.graphs, self.events = [], []
+        """CUDA graphs, one per lengths variant (the workload's step cycle):
+        the full step, and the step's decodes alone (for the decode roofline).
+        No timing events inside the graphs: an event node costs a few
+        microseconds and would break the launch chaining."""
+        self.graphs, self.decode_graphs = [], []
         for v in range(self.w.num_steps):
-            ev = [(torch.cuda.Event(enable_timing=True, external=True),
-                   torch.cuda.Event(enable_timing=True, external=True))
-                  for _ in range(self.w.num_layers)]
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                self.launch_step(stream, v, ev)
-            self.graphs.append(g)
-            self.events.append(ev)
+            for only, dst in ((False, self.graphs), (True, self.decode_graphs)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    self.launch_step(stream, v, decode_only=only)
+                dst.append(g)
 
     def replay(self, i):
         self.graphs[i % len(self.graphs)].replay()
 
-    def decode_times(self):
-        """(ms, algorithmic bytes) of every decode launch in the last replay
-        of each graph."""
-        out = []
-        for v, ev in enumerate(self.events):
-            nbytes = alg_bytes_decode(self.w.seq_lens(v + 1))
-            out += [(a.elapsed_time(b), nbytes) for a, b in ev]
-        return out
+    def replay_decodes(self, i):
+        self.decode_graphs[i % len(self.decode_graphs)].replay()
+
+    def decode_bytes(self, i):
+        """Algorithmic bytes of one decode launch of lengths variant i."""
+        return alg_bytes_decode(self.w.seq_lens(i % self.w.num_steps + 1))
 
 
 def run_ours(args, rank, world, local_rank):
@@ -237,8 +261,12 @@ def run_ours(args, rank, world, local_rank):
         r.replay(i)
     torch.cuda.synchronize()
 
-    # ---- timed region: K graph launches, one decode step each
+    # ---- timed region: (A) K full steps, then (B) the decodes of K steps
+    # alone, back to back, for the decode kernel's launch duration
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(max(args.warmup, w.num_steps)):
+        r.replay_decodes(i)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
@@ -247,13 +275,17 @@ def run_ours(args, rank, world, local_rank):
             for i in range(args.steps):
                 r.replay(i)
             t1.record(stream)
+            d0.record(stream)
+            for i in range(args.steps):
+                r.replay_decodes(i)
+            d1.record(stream)
         stream.synchronize()
         torch.cuda.synchronize()
     barrier()
     ms = t0.elapsed_time(t1)
-    times = r.decode_times()
-    dec_ms = [t for t, _ in times]
-    dec_bytes = [nb for _, nb in times]
+    dec_launches = args.steps * w.num_layers
+    avg_dec_s = max_over_ranks(d0.elapsed_time(d1), device) / dec_launches / 1e3
+    avg_bytes = sum(r.decode_bytes(i) for i in range(args.steps)) / args.steps
     err = pkv.get_device_error(r.pool, stream)
     if err != 0:
         raise RuntimeError("device error during timed region: %s" % pkv.status_string(err))
@@ -266,9 +298,8 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
     peak, peak_kind = measured_peaks()
-    avg_dec_s = sum(dec_ms) / len(dec_ms) / 1e3
-    avg_bytes = sum(dec_bytes) / len(dec_bytes)
     achieved = avg_bytes / avg_dec_s / 1e9
+    traffic = recorded_traffic(w.name, avg_bytes)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -286,15 +317,17 @@ def run_ours(args, rank, world, local_rank):
         },
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
-            "kernel": "decode_kernel", "alg_bytes_per_launch": avg_bytes,
-            "avg_launch_us": avg_dec_s * 1e6, "launches": len(dec_ms),
+            "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+            "kernel": "decode_kernel (+ split-KV merge_kernel)",
+            "alg_bytes_per_launch": avg_bytes, "avg_launch_us": avg_dec_s * 1e6,
+            "launches": dec_launches,
         },
         "decode_only_queries_per_s": w.batch / avg_dec_s,
         "e2e": e2e,
-        "gpu_launches": args.steps * w.num_layers * 3,
-        "decode_timing": "CUDA events recorded inside the step graphs, last replay of each "
-                         "of the %d graphs (%d decode launches)" % (w.num_steps, len(dec_ms)),
+        "gpu_launches": args.steps * w.num_layers * 3 + dec_launches * 2,
+        "decode_timing": "CUDA events around %d back-to-back replays of the step's decode "
+                         "launches alone (decode + merge per layer, %d launches)" %
+                         (args.steps, dec_launches),
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline:
