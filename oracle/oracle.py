@@ -23,20 +23,24 @@ class OracleError(RuntimeError):
         self.code = code
 
 
+def load(path):
+    """Open an oracle library at `path` and declare its functions."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    i32 = ctypes.c_int32
+    lib.pkvo_append.argtypes = [P, i32, P, i32, i32, i32, P, P, P, i32]
+    lib.pkvo_gather.argtypes = [P, i32, P, i32, i32, i32, P, i32, P, P, i32]
+    lib.pkvo_decode.argtypes = [P, P, i32, P, i32, i32, i32, P, i32, ctypes.c_double,
+                                P, P, i32, i32]
+    for f in (lib.pkvo_append, lib.pkvo_gather, lib.pkvo_decode):
+        f.restype = ctypes.c_int
+    return lib
+
+
 def _lib():
     global _LIB
     if _LIB is None:
-        path = _build.build()
-        lib = ctypes.CDLL(path)
-        P = ctypes.c_void_p
-        i32 = ctypes.c_int32
-        lib.pkvo_append.argtypes = [P, i32, P, i32, i32, i32, P, P, P, i32]
-        lib.pkvo_gather.argtypes = [P, i32, P, i32, i32, i32, P, i32, P, P, i32]
-        lib.pkvo_decode.argtypes = [P, P, i32, P, i32, i32, i32, P, i32, ctypes.c_double,
-                                    P, P, i32, i32]
-        for f in (lib.pkvo_append, lib.pkvo_gather, lib.pkvo_decode):
-            f.restype = ctypes.c_int
-        _LIB = lib
+        _LIB = load(_build.build())
     return _LIB
 
 
