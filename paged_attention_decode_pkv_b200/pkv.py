@@ -150,6 +150,11 @@ class Pool:
             raise RuntimeError("pool destroyed")
         return self._h
 
+    def reset_workspaces(self):
+        """Zero every cached workspace."""
+        for ws in self._ws.values():
+            ws.zero_()
+
     def close(self):
         if self._h:
             with torch.cuda.device(self.device):
@@ -180,7 +185,7 @@ class Pool:
         key = (int(batch), int(kernel), int(grid_ctas))
         ws = self._ws.get(key)
         if ws is None:
-            ws = torch.empty(max(256, self.workspace_bytes(*key)), dtype=torch.uint8,
+            ws = torch.zeros(max(256, self.workspace_bytes(*key)), dtype=torch.uint8,
                              device=self.device)
             self._ws[key] = ws
         return ws

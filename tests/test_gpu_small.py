@@ -34,11 +34,13 @@ def test_decode_edge_lengths(kernel, lens):
 
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("grid,min_chunk", [(1, 0), (2, 0), (7, 0), (3, 1), (0, 1), (0, 3),
-                                            (0, 64), (50, 2), (100, 1), (77, 0)])
+                                            (0, 64), (50, 2), (100, 1), (77, 0), (400, 1),
+                                            (600, 0)])
 def test_decode_split_patterns(kernel, grid, min_chunk):
-    # Different grids / chunk sizes cut the (sequence, kv head) runs at
+    # Different grids / chunk sizes cut the sequences' page runs at
     # different places, exercising the split-KV merge; the result must stay
-    # within tolerance of the oracle for every cut.
+    # within tolerance of the oracle for every cut, including grids (400,
+    # 600 CTAs) larger than the device holds at once.
     g = GpuCase(make_case([300, 1, 47, 129, 16, 517], seed=77, spare_pages=9))
     want = g.oracle(scale=0.09)
     got = g.decode(scale=0.09, kernel=kernel, grid_ctas=grid, min_chunk=min_chunk)
