@@ -371,34 +371,43 @@ def run_e2e(r: Runner, stream, steps, device, world):
 
 # ------------------------------------------------------------ oracle arms --
 
-def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None):
-    """Time the FP64 oracle on whole-layer decodes of step 1 (all sequences
-    of the batch), layer after layer, until ``max_seconds`` have passed.
-    Returns (queries, seconds, threads, layers_done)."""
+def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None, max_layers=None):
+    """Time the FP64 oracle on whole-layer append + decode of step 1 (all
+    sequences of the batch), cycling over `layers`, until `max_seconds` of
+    oracle time have passed (at least one layer; at most `max_layers`).
+    Each layer's pages are copied to the host once and re-copied (host side)
+    before every repeat, outside the timed part.  Returns (queries, seconds,
+    threads, layer-decodes done)."""
     import oracle
-    layers = list(range(w.num_layers)) if layers is None else layers
+    layers = list(range(w.num_layers)) if layers is None else list(layers)
     threads = os.cpu_count() or 1
     sl = w.seq_lens(1)
+    cache = {}
     done, secs = 0, 0.0
-    for l in layers:
-        pool_h, bt_h = W.compact_pages(w, pool_t, range(w.batch), [l])
-        q, k, v = W.step_inputs(w, 1, l, pool_t.device)
-        qb, kb, vb = W.bits(q), W.bits(k), W.bits(v)
+    while True:
+        l = layers[done % len(layers)]
+        if l not in cache:
+            pool_h, bt_h = W.compact_pages(w, pool_t, range(w.batch), [l])
+            q, k, v = W.step_inputs(w, 1, l, pool_t.device)
+            cache[l] = (pool_h, bt_h, W.bits(q), W.bits(k), W.bits(v))
+        pool_h0, bt_h, qb, kb, vb = cache[l]
+        pool_h = pool_h0.copy()
         t = time.perf_counter()
         oracle.append(pool_h, bt_h, sl, kb, vb, l)
         oracle.decode(qb, pool_h, bt_h, sl, l, w.scale, nthreads=threads)
         secs += time.perf_counter() - t
         done += 1
-        if secs >= max_seconds:
+        if secs >= max_seconds or (max_layers is not None and done >= max_layers):
             break
     return done * w.batch, secs, threads, done
 
 
 def cpu_baseline(w, pool_t, max_seconds):
-    q, s, thr, layers = oracle_sample(w, pool_t, max_seconds)
+    q, s, thr, layers = oracle_sample(w, pool_t, max_seconds, max_layers=4096)
     return {"value": q / s, "unit": UNIT, "cores": thr, "kind": "oracle",
-            "sample": "%d whole-layer append+decode(s) of step 1 (%d sequences each), "
-                      "%.1f s of FP64 oracle work" % (layers, w.batch, s)}
+            "sample": "%d whole-layer append+decode(s) of step 1, cycling over the %d layers "
+                      "(%d sequences each), %.1f s of FP64 oracle work" %
+                      (layers, w.num_layers, w.batch, s)}
 
 
 def run_reference(args, rank, world, local_rank):
@@ -413,11 +422,11 @@ def run_reference(args, rank, world, local_rank):
     pool_t = W.make_pool(w, dev)
     nl = w.num_layers
     for i in range(args.warmup):
-        oracle_sample(w, pool_t, 0.0, layers=[i % nl])
+        oracle_sample(w, pool_t, 0.0, layers=[i % nl], max_layers=1)
     q_tot, s_tot = 0, 0.0
     thr = 1
     for i in range(args.steps):
-        q, s, thr, _ = oracle_sample(w, pool_t, 0.0, layers=[i % nl])
+        q, s, thr, _ = oracle_sample(w, pool_t, 0.0, layers=[i % nl], max_layers=1)
         q_tot += q
         s_tot += s
     v = q_tot / s_tot
