@@ -30,6 +30,8 @@ def load(path):
     i32 = ctypes.c_int32
     lib.pkvo_append.argtypes = [P, i32, P, i32, i32, i32, P, P, P, i32]
     lib.pkvo_gather.argtypes = [P, i32, P, i32, i32, i32, P, i32, P, P, i32]
+    lib.pkvo_fill.argtypes = [P, i32, P, i32, i32, i32, P, P, P, P, i32]
+    lib.pkvo_fill.restype = ctypes.c_int
     lib.pkvo_decode.argtypes = [P, P, i32, P, i32, i32, i32, P, i32, ctypes.c_double,
                                 P, P, i32, i32]
     for f in (lib.pkvo_append, lib.pkvo_gather, lib.pkvo_decode):
@@ -71,6 +73,20 @@ def append(pool, block_tables, seq_lens, k_new, v_new, layer):
     L, B, MB = bt.shape
     _check(_lib().pkvo_append(_p(pool), pool.shape[0], _p(bt), L, B, MB, _p(sl), _p(k), _p(v),
                               int(layer)))
+
+
+def fill(pool, block_tables, cu, start, k_src, v_src, layer):
+    """In-place prefill write of a ragged token batch (see pkv_oracle.h)."""
+    if not (pool.flags.c_contiguous and pool.dtype == np.uint16):
+        raise TypeError("pool must be C-contiguous uint16")
+    bt = _c(block_tables, np.int32)
+    cu = _c(cu, np.int32)
+    st = _c(start, np.int32)
+    k = _c(k_src, np.uint16)
+    v = _c(v_src, np.uint16)
+    L, B, MB = bt.shape
+    _check(_lib().pkvo_fill(_p(pool), pool.shape[0], _p(bt), L, B, MB, _p(cu), _p(st), _p(k),
+                            _p(v), int(layer)))
 
 
 def gather(pool, block_tables, seq_lens, layer, max_seq_len, k_out=None, v_out=None):

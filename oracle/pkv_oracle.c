@@ -83,6 +83,42 @@ int pkvo_append(uint16_t *pool, int32_t num_pages, const int32_t *block_tables,
   return PKVO_OK;
 }
 
+int pkvo_fill(uint16_t *pool, int32_t num_pages, const int32_t *block_tables,
+              int32_t num_layers, int32_t batch, int32_t max_blocks, const int32_t *cu,
+              const int32_t *start, const uint16_t *k_src, const uint16_t *v_src,
+              int32_t layer) {
+  /* Prefill writes a request's tokens into its pages (comrad404 article on
+   * samir-vllm, section "Что README говорит о KV-кэше и пакетном
+   * декодировании"), token by token through the block table. */
+  if (!pool || !block_tables || !cu || !start || !k_src || !v_src) return PKVO_BAD_ARG;
+  if (batch < 0 || max_blocks < 0 || num_pages < 0) return PKVO_BAD_ARG;
+  if (layer < 0 || layer >= num_layers) return PKVO_BAD_ARG;
+  if (batch > 0 && cu[0] != 0) return PKVO_BAD_ARG;
+  for (int32_t b = 0; b < batch; ++b) {
+    if (cu[b + 1] < cu[b] || start[b] < 0) return PKVO_BAD_ARG;
+    int64_t end = (int64_t)start[b] + (cu[b + 1] - cu[b]);
+    if (end > (int64_t)max_blocks * O_TOKENS_PER_PAGE) return PKVO_BAD_LEN;
+    for (int64_t pos = start[b]; pos < end; ++pos)
+      if (o_page_of(block_tables, batch, max_blocks, layer, b, pos, num_pages) < 0)
+        return PKVO_BAD_PAGE;
+  }
+  for (int32_t b = 0; b < batch; ++b) {
+    for (int32_t i = 0; i < cu[b + 1] - cu[b]; ++i) {
+      int64_t pos = (int64_t)start[b] + i;
+      int64_t page = o_page_of(block_tables, batch, max_blocks, layer, b, pos, num_pages);
+      int slot = (int)(pos % O_TOKENS_PER_PAGE);
+      for (int g = 0; g < O_KV_HEADS; ++g) {
+        for (int d = 0; d < O_DIM; ++d) {
+          int64_t src = ((int64_t)(cu[b] + i) * O_KV_HEADS + g) * O_DIM + d;
+          pool[o_offset(page, 0, g, slot, d)] = k_src[src];
+          pool[o_offset(page, 1, g, slot, d)] = v_src[src];
+        }
+      }
+    }
+  }
+  return PKVO_OK;
+}
+
 int pkvo_gather(const uint16_t *pool, int32_t num_pages,
                 const int32_t *block_tables, int32_t num_layers, int32_t batch,
                 int32_t max_blocks, const int32_t *seq_lens, int32_t layer,

@@ -64,6 +64,17 @@ int pkvo_append(uint16_t *pool, int32_t num_pages, const int32_t *block_tables,
                 const int32_t *seq_lens, const uint16_t *k_new,
                 const uint16_t *v_new, int32_t layer);
 
+/* Fill (prefill, or chunked prefill): sequence b writes its tokens
+ * k_src/v_src[cu[b] + i][g][:], i < cu[b+1] - cu[b], at positions
+ * start[b] + i, each into slot pos % 16 of page block_tables[layer][b][pos/16]
+ * (the prefill half of "prefill fills the request's pages, decode adds the
+ * new token", comrad404 article, KV-cache section).  k_src / v_src are
+ * [cu[batch]][8][64].  Checks every token before writing anything. */
+int pkvo_fill(uint16_t *pool, int32_t num_pages, const int32_t *block_tables,
+              int32_t num_layers, int32_t batch, int32_t max_blocks, const int32_t *cu,
+              const int32_t *start, const uint16_t *k_src, const uint16_t *v_src,
+              int32_t layer);
+
 /* Gather: k_out[b][g][t][d] = K of token t of sequence b (and likewise V),
  * for t < seq_lens[b]; entries t >= seq_lens[b] are left untouched.
  * k_out / v_out are [batch][8][max_seq_len][64]. */

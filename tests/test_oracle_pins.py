@@ -251,3 +251,56 @@ def test_decode_rejects_bad_page_and_length():
         oracle.decode(c["q"], c["pool"], bad, c["seq_lens"], 0, 0.125)
     with pytest.raises(oracle.OracleError):
         oracle.decode(c["q"], c["pool"], c["bt"], np.array([17, 10_000], np.int32), 0, 0.125)
+
+
+# -------------------------------------------------------------------- fill --
+
+def _ragged(rng, lens_before, counts):
+    cu = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    k = bf16_bits(rng.standard_normal((int(cu[-1]), G, D)))
+    v = bf16_bits(rng.standard_normal((int(cu[-1]), G, D)))
+    return cu, np.asarray(lens_before, np.int32), k, v
+
+
+def test_fill_equals_successive_appends():
+    # A prefill of T tokens is T appends in a row (the append index is
+    # pinned above), so both must leave the same pool bits.
+    lens_after = [37, 16, 5, 50]
+    c = make_case(lens_after, seed=61, spare_pages=4)
+    rng = np.random.default_rng(4)
+    start = [3, 0, 5, 20]
+    counts = [34, 16, 0, 30]
+    cu, st, k, v = _ragged(rng, start, counts)
+    filled = c["pool"].copy()
+    oracle.fill(filled, c["bt"], cu, st, k, v, 0)
+    appended = c["pool"].copy()
+    for i in range(max(counts)):
+        rows = [b for b in range(4) if i < counts[b]]
+        if not rows:
+            continue
+        sl = np.array([st[b] + i + 1 for b in rows], np.int32)
+        bt = c["bt"][:, rows, :]
+        oracle.append(appended, bt, sl, k[[cu[b] + i for b in rows]], v[[cu[b] + i for b in rows]], 0)
+    assert np.array_equal(filled, appended)
+
+
+def test_fill_then_gather_returns_the_tokens():
+    c = make_case([40, 17], seed=67, spare_pages=2)
+    rng = np.random.default_rng(5)
+    cu, st, k, v = _ragged(rng, [0, 0], [40, 17])
+    pool = np.full_like(c["pool"], NAN)
+    oracle.fill(pool, c["bt"], cu, st, k, v, 0)
+    ko, vo = oracle.gather(pool, c["bt"], c["seq_lens"], 0, 40)
+    for b, n in enumerate([40, 17]):
+        assert np.array_equal(ko[b, :, :n].transpose(1, 0, 2), k[cu[b]:cu[b + 1]])
+        assert np.array_equal(vo[b, :, :n].transpose(1, 0, 2), v[cu[b]:cu[b + 1]])
+
+
+def test_fill_rejects_out_of_range_without_writing():
+    c = make_case([20, 5], seed=71)
+    rng = np.random.default_rng(6)
+    cu, st, k, v = _ragged(rng, [10, 0], [40, 5])    # 10 + 40 > max_blocks * 16 = 32
+    pool = c["pool"].copy()
+    with pytest.raises(oracle.OracleError):
+        oracle.fill(pool, c["bt"], cu, st, k, v, 0)
+    assert np.array_equal(pool, c["pool"])
