@@ -295,6 +295,9 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API from pinned host buffers
     e2e = run_e2e(r, stream, min(args.steps, args.e2e_steps), device, world)
 
+    # ---- prefill page fill bandwidth (rewrites the prompt tokens' values)
+    fill = None if args.no_fill else run_fill(r, stream, min(args.steps, 50), device)
+
     if rank != 0:
         return None
     peak, peak_kind = measured_peaks()
@@ -324,6 +327,7 @@ def run_ours(args, rank, world, local_rank):
         },
         "decode_only_queries_per_s": w.batch / avg_dec_s,
         "e2e": e2e,
+        "prefill_fill": fill,
         "gpu_launches": args.steps * w.num_layers * 3 + dec_launches * 2,
         "decode_timing": "CUDA events around %d back-to-back replays of the step's decode "
                          "launches alone (decode + merge per layer, %d launches)" %
@@ -367,6 +371,68 @@ def run_e2e(r: Runner, stream, steps, device, world):
     return {"value": whole_job_rate(steps * w.num_layers * w.batch, world, ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps}
+
+
+def run_fill(r: Runner, stream, steps, device):
+    """Prefill page fill (pkv_fill) of every sequence's prompt, all layers:
+    one CUDA graph of num_layers fill launches, each from its own source
+    buffer into that layer's pages, so a step moves far more than L2 holds.
+    Algorithmic bytes per launch: each prompt token's K and V read once and
+    written once (2 x 2048 B)."""
+    pkv = r.pkv
+    w = r.w
+    counts = w.prefill_lens.astype(np.int64)
+    T = int(counts.sum())
+    if T == 0:
+        return None
+    cu = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(device)
+    start = torch.zeros(w.batch, dtype=torch.int32, device=device)
+    per_layer = 2 * T * 2048
+    nbuf = max(1, min(w.num_layers, (8 << 30) // per_layer))
+    gen = torch.Generator(device=device)
+    gen.manual_seed(1234)
+    src = [(torch.randn((T, 8, 64), generator=gen, device=device).to(torch.bfloat16),
+            torch.randn((T, 8, 64), generator=gen, device=device).to(torch.bfloat16))
+           for _ in range(nbuf)]
+
+    def launch():
+        for l in range(w.num_layers):
+            k, v = src[l % nbuf]
+            pkv.fill(r.pool, r.bt, cu, start, k, v, l, stream=stream)
+
+    with torch.cuda.stream(stream):
+        launch()
+    stream.synchronize()
+    if pkv.get_device_error(r.pool, stream) != 0:
+        raise RuntimeError("device error in pkv_fill")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        launch()
+    for _ in range(3):
+        g.replay()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        t1.record(stream)
+    stream.synchronize()
+    barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1), device)
+    if pkv.get_device_error(r.pool, stream) != 0:
+        raise RuntimeError("device error in pkv_fill")
+    launches = steps * w.num_layers
+    avg_s = ms / launches / 1e3
+    peak, peak_kind = measured_peaks()
+    achieved = per_layer / avg_s / 1e9
+    return {"kernel": "fill_kernel", "tokens_per_launch": T, "alg_bytes_per_launch": per_layer,
+            "avg_launch_us": avg_s * 1e6, "launches": launches, "achieved": achieved,
+            "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+            "source_buffers": nbuf,
+            "timing": "CUDA events around %d replays of one graph of %d fill launches" %
+                      (steps, w.num_layers)}
 
 
 # ------------------------------------------------------------ oracle arms --
@@ -456,6 +522,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fill", action="store_true", help="skip the prefill fill timing")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch")
     args = ap.parse_args()

@@ -81,12 +81,12 @@ typedef enum {
   PKV_ERR_INVALID_ARG = -1,    /* null pointer, negative size, layer out of range  */
   PKV_ERR_UNSUPPORTED = -2,    /* shape other than 16 tokens / 8 kv heads / d 64    */
   PKV_ERR_CUDA = -3,           /* a CUDA runtime call failed                        */
-  PKV_ERR_OUT_OF_PAGES = -4,   /* reserved for page allocators built on this ABI    */
+  PKV_ERR_OUT_OF_PAGES = -4,   /* page allocator: not enough free pages right now    */
   PKV_ERR_BAD_PAGE = -5,       /* device: block-table entry outside [0, num_pages)  */
   PKV_ERR_WORKSPACE = -6,      /* workspace missing, misaligned or too small        */
   PKV_ERR_DEVICE_TIMEOUT = -7, /* device: a bounded wait on a copy ran out           */
   PKV_ERR_BAD_SEQ_LEN = -8,    /* device: seq_len < 0 (append: < 1) or too long      */
-  PKV_ERR_TOO_LARGE = -9       /* batch too large for the fixed no-alloc scratch     */
+  PKV_ERR_TOO_LARGE = -9       /* larger than the no-alloc scratch / the whole pool */
 } pkv_status;
 
 /* Launch flags for pkv_pool_set_launch_flags. */
@@ -161,6 +161,52 @@ PKV_API int pkv_pool_set_launch_flags(pkv_pool *pool, int32_t flags);
 PKV_API int pkv_append(pkv_pool *pool, const int32_t *block_tables, const int32_t *seq_lens,
                const uint16_t *k_new, const uint16_t *v_new, int32_t layer,
                int32_t num_layers, int32_t batch, int32_t max_blocks, pkv_stream_t stream);
+
+/*
+ * Fill (prefill, or chunked prefill): the counterpart of pkv_append for many
+ * tokens; prefill is the step that fills a request's pages (comrad404 article
+ * on samir-vllm, section "Что README говорит о KV-кэше и пакетном
+ * декодировании").  Sequence b writes its tokens k_src/v_src[cu_tokens[b] +
+ * i][g][:], i < cu_tokens[b+1] - cu_tokens[b], at positions start_pos[b] + i,
+ * each in slot pos % 16 of page block_tables[layer][b][pos / 16].  Bit
+ * copies.  k_src, v_src: dev BF16 [total_tokens][8][64], 16-byte aligned
+ * (NULL allowed when total_tokens is 0); total_tokens: host int, the row
+ * count of k_src and v_src, which sizes the grid (0 launches nothing);
+ * cu_tokens: dev int32 [batch+1], from 0, non-decreasing, ending at
+ * total_tokens; start_pos: dev int32 [batch].  Device errors
+ * (PKV_ERR_BAD_SEQ_LEN): cu_tokens[0] != 0 or cu_tokens[batch] !=
+ * total_tokens (nothing written), a decreasing entry (reported; which tokens
+ * are written is then unspecified), a negative start or a position beyond
+ * max_blocks*16 (that sequence is skipped).  A page outside the pool ->
+ * PKV_ERR_BAD_PAGE (that token is skipped).  Whatever the device inputs, no
+ * source row outside [0, total_tokens) is read and nothing outside the pool
+ * is written.  The positions of different sequences must name different
+ * slots.  Stream ordered; PDL-chained like pkv_append when the pool's PDL
+ * flag is set.  max_blocks * 16 must fit in int32.
+ */
+PKV_API int pkv_fill(pkv_pool *pool, const int32_t *block_tables, const int32_t *cu_tokens,
+                     const int32_t *start_pos, const uint16_t *k_src, const uint16_t *v_src,
+                     int32_t total_tokens, int32_t layer, int32_t num_layers, int32_t batch,
+                     int32_t max_blocks, pkv_stream_t stream);
+
+/*
+ * Host page allocator (no GPU work; not thread-safe).  Hands out physical
+ * page ids of a pool of num_pages pages from a LIFO free stack (page 0 first
+ * on a fresh allocator), all or nothing:
+ *  - pkv_allocator_alloc(count): PKV_ERR_TOO_LARGE if count exceeds the whole
+ *    pool (such a request can never run: reject it), PKV_ERR_OUT_OF_PAGES if
+ *    fewer than count pages are free now (queue the request, first in first
+ *    out, and retry when pages are freed); nothing is taken on error.
+ *  - pkv_allocator_free(pages, count): returns pages (for instance when a
+ *    sequence ends); PKV_ERR_INVALID_ARG, and nothing freed, if a page is out
+ *    of range, not allocated, or listed twice.
+ */
+typedef struct pkv_page_allocator pkv_page_allocator;
+PKV_API int pkv_allocator_create(int32_t num_pages, pkv_page_allocator **out);
+PKV_API int pkv_allocator_destroy(pkv_page_allocator *alloc);
+PKV_API int32_t pkv_allocator_free_count(const pkv_page_allocator *alloc);
+PKV_API int pkv_allocator_alloc(pkv_page_allocator *alloc, int32_t count, int32_t *pages_out);
+PKV_API int pkv_allocator_free(pkv_page_allocator *alloc, const int32_t *pages, int32_t count);
 
 /*
  * Workspace bytes paged_attention_decode needs for this batch on the pool's

@@ -11,7 +11,11 @@
 // pages in place); the gather exists so that page indexing can be checked
 // bit for bit.
 //
-// Both are pure 16-byte copies: 8 consecutive threads move one 128-byte row
+// Fill: the prefill counterpart of append -- prefill writes a request's
+// prompt tokens into its pages (same comrad404 section) -- a ragged batch of
+// tokens per sequence, written at consecutive positions from start_pos[b].
+//
+// All three are pure 16-byte copies: 8 consecutive threads move one 128-byte row
 // (one token of one kv head), so every warp access is four full 128-byte
 // lines.
 #include "pkv_internal.cuh"
@@ -51,6 +55,88 @@ __global__ void __launch_bounds__(128) append_kernel(const uint4* __restrict__ k
   const int64_t row = (static_cast<int64_t>(phys) * 2 + kv) * (kKvHeads * kTokens) +
                       g * kTokens + slot;
   pool[row * 8 + c] = *src;
+}
+
+// Fill: one CTA per kFillRowsPerCta consecutive source rows t (rows
+// [0, total) of k_src / v_src).  512 threads = 4 row lanes x (K|V) x 8 kv
+// heads x 8 chunks of 16 B; each lane moves kFillRowsPerLane rows, with all
+// its loads issued first.  While they are in flight, one thread per row maps
+// the row to its destination -- row t belongs to the last sequence b with
+// cu[b] <= t (binary search over cu), goes to position start[b] + t - cu[b],
+// so to slot pos % 16 of page bt[b][pos / 16] -- and shares it through
+// shared memory: the index loads are issued once per row, not once per
+// 16-byte chunk.  The grid follows the row count, not (sequence x longest
+// prompt), so a batch of mixed prompt lengths launches no empty CTAs.
+constexpr int kFillThreads = 512;
+constexpr int kFillLanes = kFillThreads / 128;
+constexpr int kFillRowsPerLane = 4;
+constexpr int kFillRowsPerCta = kFillLanes * kFillRowsPerLane;
+
+__device__ __forceinline__ int32_t fill_seq_of(const int32_t* __restrict__ cu, int32_t batch,
+                                               int32_t t) {
+  int32_t lo = 0, hi = batch;   // cu[lo] <= t < cu[hi] when cu is non-decreasing
+  while (hi - lo > 1) {
+    const int32_t mid = (lo + hi) >> 1;
+    if (cu[mid] <= t) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kFillThreads)
+    fill_kernel(const uint4* __restrict__ k_src, const uint4* __restrict__ v_src,
+                uint4* __restrict__ pool, const int32_t* __restrict__ bt,
+                const int32_t* __restrict__ cu, const int32_t* __restrict__ start,
+                int32_t* __restrict__ err, int32_t batch, int32_t max_blocks,
+                int32_t num_pages, int32_t total) {
+  __shared__ int64_t s_row[kFillRowsPerCta];   // pool row of (page, K, head 0, slot), or -1
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  const int kv = (tid >> 6) & 1;
+  const int g = (tid >> 3) & 7;
+  const int c = tid & 7;
+  // the rows the caller passed must be exactly the rows cu describes
+  if (cu[0] != 0 || cu[batch] != total) {   // uniform over the grid
+    if (blockIdx.x == 0 && tid == 0) record_error(err, kErrBadLen);
+    return;
+  }
+  // a decreasing cu makes the row -> sequence map ambiguous: report it
+  for (int32_t b = blockIdx.x * blockDim.x + tid; b < batch; b += gridDim.x * blockDim.x)
+    if (cu[b + 1] < cu[b]) record_error(err, kErrBadLen);
+  const int32_t row0 = blockIdx.x * kFillRowsPerCta;
+  const uint4* src = kv ? v_src : k_src;
+  uint4 val[kFillRowsPerLane];
+#pragma unroll
+  for (int j = 0; j < kFillRowsPerLane; ++j) {
+    const int32_t t = row0 + (tid >> 7) + kFillLanes * j;
+    if (t < total) val[j] = __ldcs(src + (static_cast<int64_t>(t) * kKvHeads + g) * 8 + c);
+  }
+  if (tid < kFillRowsPerCta) {
+    const int32_t t = row0 + tid;
+    int64_t row = -1;
+    if (t < total) {
+      const int32_t b = fill_seq_of(cu, batch, t);
+      const int32_t c0 = cu[b], c1 = cu[b + 1], s0 = start[b];
+      if (t < c0 || t >= c1 || s0 < 0 ||
+          static_cast<int64_t>(s0) + (c1 - c0) > static_cast<int64_t>(max_blocks) * kTokens) {
+        record_error(err, kErrBadLen);
+      } else {
+        const int32_t pos = s0 + (t - c0);
+        const int32_t phys = bt[static_cast<int64_t>(b) * max_blocks + pos / kTokens];
+        if (phys < 0 || phys >= num_pages)
+          record_error(err, kErrBadPage);
+        else
+          row = static_cast<int64_t>(phys) * (2 * kKvHeads * kTokens) + pos % kTokens;
+      }
+    }
+    s_row[tid] = row;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kFillRowsPerLane; ++j) {
+    const int64_t row = s_row[(tid >> 7) + kFillLanes * j];
+    if (row >= 0) pool[(row + (kv * kKvHeads + g) * kTokens) * 8 + c] = val[j];
+  }
 }
 
 // grid (ceil(max_seq_len / 32), 8 kv heads, batch); 256 threads = 32 tokens
@@ -103,6 +189,25 @@ cudaError_t launch_append(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new
   return cudaLaunchKernelEx(&cfg, append_kernel, reinterpret_cast<const uint4*>(k_new),
                             reinterpret_cast<const uint4*>(v_new), reinterpret_cast<uint4*>(pool),
                             bt, seq_lens, err, max_blocks, num_pages);
+}
+
+cudaError_t launch_fill(const __nv_bfloat16* k_src, const __nv_bfloat16* v_src,
+                        __nv_bfloat16* pool, const int32_t* bt, const int32_t* cu,
+                        const int32_t* start, int32_t* err, int32_t batch, int32_t max_blocks,
+                        int32_t num_pages, int32_t total_tokens, int flags, cudaStream_t stream) {
+  if (batch == 0 || total_tokens == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((total_tokens + kFillRowsPerCta - 1) / kFillRowsPerCta);
+  cfg.blockDim = dim3(kFillThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, fill_kernel, reinterpret_cast<const uint4*>(k_src),
+                            reinterpret_cast<const uint4*>(v_src), reinterpret_cast<uint4*>(pool),
+                            bt, cu, start, err, batch, max_blocks, num_pages, total_tokens);
 }
 
 cudaError_t launch_gather(const __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,

@@ -184,6 +184,25 @@ int pkv_append(pkv_pool* pool, const int32_t* block_tables, const int32_t* seq_l
       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int pkv_fill(pkv_pool* pool, const int32_t* block_tables, const int32_t* cu_tokens,
+             const int32_t* start_pos, const uint16_t* k_src, const uint16_t* v_src,
+             int32_t total_tokens, int32_t layer, int32_t num_layers, int32_t batch,
+             int32_t max_blocks, pkv_stream_t stream) {
+  int s = check_table_args(pool, block_tables, cu_tokens, layer, num_layers, batch, max_blocks);
+  if (s != PKV_OK) return s;
+  if (!start_pos || total_tokens < 0) return PKV_ERR_INVALID_ARG;
+  // the sources may be NULL only when there is no row to read
+  if (total_tokens > 0 && (!k_src || !v_src || !aligned(k_src, 16) || !aligned(v_src, 16)))
+    return PKV_ERR_INVALID_ARG;
+  // positions are int32 on the device
+  if (static_cast<int64_t>(max_blocks) * pkv::kTokens > 2147483647) return PKV_ERR_UNSUPPORTED;
+  return from_cuda(pkv::launch_fill(
+      reinterpret_cast<const __nv_bfloat16*>(k_src), reinterpret_cast<const __nv_bfloat16*>(v_src),
+      static_cast<__nv_bfloat16*>(pool->data), layer_slab(block_tables, layer, batch, max_blocks),
+      cu_tokens, start_pos, pool->d_err, batch, max_blocks, pool->num_pages, total_tokens,
+      pool->launch_flags, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int pkv_pool_set_launch_flags(pkv_pool* pool, int32_t flags) {
   if (!pool || (flags & ~(PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES | PKV_LAUNCH_TEST_STALL)))
     return PKV_ERR_INVALID_ARG;
@@ -357,7 +376,7 @@ const char* pkv_status_string(int status) {
     case PKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case PKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case PKV_ERR_BAD_SEQ_LEN: return "sequence length out of range";
-    case PKV_ERR_TOO_LARGE: return "request larger than the fixed no-alloc scratch";
+    case PKV_ERR_TOO_LARGE: return "request larger than the fixed no-alloc scratch or the whole pool";
     default: return "unknown status";
   }
 }

@@ -226,6 +226,12 @@ cudaError_t launch_append(const __nv_bfloat16* k_new, const __nv_bfloat16* v_new
                           int32_t* err, int32_t batch, int32_t max_blocks, int32_t num_pages,
                           int flags, cudaStream_t stream);
 
+cudaError_t launch_fill(const __nv_bfloat16* k_src, const __nv_bfloat16* v_src,
+                        __nv_bfloat16* pool, const int32_t* bt, const int32_t* cu,
+                        const int32_t* start, int32_t* err, int32_t batch, int32_t max_blocks,
+                        int32_t num_pages, int32_t total_tokens, int flags,
+                        cudaStream_t stream);
+
 cudaError_t launch_gather(const __nv_bfloat16* pool, const int32_t* bt, const int32_t* seq_lens,
                           __nv_bfloat16* k_out, __nv_bfloat16* v_out, int32_t* err,
                           int32_t batch, int32_t max_blocks, int32_t num_pages,

@@ -1,7 +1,8 @@
 """Python binding of libpkv (the C ABI in include/pkv.h).
 
-Argument marshalling only: every step of append, gather and decode runs in
-the CUDA kernels of libpkv.so.  Tensors are torch CUDA tensors; torch is used
+Argument marshalling only: every step of append, fill, gather and decode
+runs in the CUDA kernels of libpkv.so (the page allocator is host C code in
+the same library).  Tensors are torch CUDA tensors; torch is used
 for device memory and streams, nothing else.  There is no CPU fallback: if
 libpkv.so is missing or cannot be loaded, importing this module raises.
 """
@@ -44,6 +45,8 @@ EXPORTS = (
     "pkv_decode_workspace_bytes", "pkv_decode_workspace_bytes_ex", "paged_attention_decode",
     "paged_attention_decode_ex", "pkv_gather", "pkv_get_device_error", "pkv_status_string",
     "pkv_last_error_message", "pkv_pool_set_launch_flags", "paged_attention_decode_noalloc",
+    "pkv_fill", "pkv_allocator_create", "pkv_allocator_destroy", "pkv_allocator_free_count",
+    "pkv_allocator_alloc", "pkv_allocator_free",
 )
 
 
@@ -72,6 +75,12 @@ def _load():
         "pkv_pool_set_launch_flags": ([P, i32], ctypes.c_int),
         "paged_attention_decode_noalloc": ([P, P, P, P, i32, ctypes.c_float, P, i32, i32, i32, P],
                                            ctypes.c_int),
+        "pkv_fill": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P], ctypes.c_int),
+        "pkv_allocator_create": ([i32, ctypes.POINTER(P)], ctypes.c_int),
+        "pkv_allocator_destroy": ([P], ctypes.c_int),
+        "pkv_allocator_free_count": ([P], i32),
+        "pkv_allocator_alloc": ([P, i32, ctypes.POINTER(i32)], ctypes.c_int),
+        "pkv_allocator_free": ([P, ctypes.POINTER(i32), i32], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -236,6 +245,61 @@ def decode_noalloc(q: torch.Tensor, pool: Pool, block_tables: torch.Tensor,
         _dev(out, torch.float32, (B, NUM_Q_HEADS, HEAD_DIM), "out"), L, B, MB, _stream(stream)),
         "paged_attention_decode_noalloc")
     return out
+
+
+def fill(pool: Pool, block_tables: torch.Tensor, cu_tokens: torch.Tensor,
+         start_pos: torch.Tensor, k_src: torch.Tensor, v_src: torch.Tensor, layer: int,
+         stream=None):
+    """Write a ragged batch of tokens into the pages (prefill): sequence b's
+    tokens k_src/v_src[cu_tokens[b]:cu_tokens[b+1]] go to positions
+    start_pos[b], start_pos[b]+1, ..."""
+    L, B, MB = block_tables.shape
+    T = k_src.shape[0]
+    _check(lib.pkv_fill(pool.handle, _dev(block_tables, torch.int32, None, "block_tables"),
+                        _dev(cu_tokens, torch.int32, (B + 1,), "cu_tokens"),
+                        _dev(start_pos, torch.int32, (B,), "start_pos"),
+                        _dev(k_src, torch.bfloat16, (T, NUM_KV_HEADS, HEAD_DIM), "k_src"),
+                        _dev(v_src, torch.bfloat16, (T, NUM_KV_HEADS, HEAD_DIM), "v_src"),
+                        T, int(layer), L, B, MB, _stream(stream)), "pkv_fill")
+
+
+class PageAllocator:
+    """Host page allocator over page ids 0..num_pages-1 (pkv_allocator_*).
+
+    alloc(n) returns n page ids or raises PkvError with status
+    ERR_OUT_OF_PAGES (not enough free now: wait) or ERR_TOO_LARGE (more than
+    the whole pool: reject); free(pages) returns them."""
+
+    def __init__(self, num_pages: int):
+        h = ctypes.c_void_p()
+        _check(lib.pkv_allocator_create(int(num_pages), ctypes.byref(h)), "pkv_allocator_create")
+        self.handle = h
+        self.num_pages = int(num_pages)
+
+    @property
+    def free_count(self) -> int:
+        return int(lib.pkv_allocator_free_count(self.handle))
+
+    def alloc(self, count: int) -> list:
+        buf = (ctypes.c_int32 * max(int(count), 1))()
+        _check(lib.pkv_allocator_alloc(self.handle, int(count), buf), "pkv_allocator_alloc")
+        return list(buf[:int(count)])
+
+    def free(self, pages) -> None:
+        pages = [int(p) for p in pages]
+        buf = (ctypes.c_int32 * max(len(pages), 1))(*pages)
+        _check(lib.pkv_allocator_free(self.handle, buf, len(pages)), "pkv_allocator_free")
+
+    def close(self):
+        if self.handle:
+            lib.pkv_allocator_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def gather(pool: Pool, block_tables: torch.Tensor, seq_lens: torch.Tensor, layer: int,

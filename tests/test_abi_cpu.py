@@ -65,3 +65,4 @@ def test_calls_reject_null_pool():
     assert pkv.lib.pkv_decode_workspace_bytes(None, 4, ctypes.byref(n)) == pkv.ERR_INVALID_ARG
     assert pkv.lib.pkv_pool_destroy(None) == pkv.OK
     assert pkv.lib.pkv_pool_num_pages(None) == -1
+    assert pkv.lib.pkv_fill(None, P, P, P, P, P, 16, 0, 1, 1, 1, None) == pkv.ERR_INVALID_ARG

@@ -23,8 +23,14 @@ MUTANTS = {
     "scores_from_values": ("o_bf16(jb->pool[o_offset(page, 0, g, slot, d)])",
                            "o_bf16(jb->pool[o_offset(page, 1, g, slot, d)])"),
     "weights_not_per_token": ("oh[d] += w[t] * o_bf16", "oh[d] += w[0] * o_bf16"),
-    "append_wrong_slot": ("int slot = (int)(pos % O_TOKENS_PER_PAGE);",
-                          "int slot = (int)((pos + 1) % O_TOKENS_PER_PAGE);"),
+    "append_wrong_slot": ("int slot = (int)(pos % O_TOKENS_PER_PAGE);\n    for",
+                          "int slot = (int)((pos + 1) % O_TOKENS_PER_PAGE);\n    for"),
+    "fill_wrong_slot": ("int slot = (int)(pos % O_TOKENS_PER_PAGE);\n      for",
+                        "int slot = (int)((pos + 1) % O_TOKENS_PER_PAGE);\n      for"),
+    "fill_source_row_not_offset": ("((int64_t)(cu[b] + i) * O_KV_HEADS + g)",
+                                   "((int64_t)(i) * O_KV_HEADS + g)"),
+    "fill_v_from_k": ("pool[o_offset(page, 1, g, slot, d)] = v_src[src];",
+                      "pool[o_offset(page, 1, g, slot, d)] = k_src[src];"),
     "gather_k_from_v": ("k_out[dst] = pool[o_offset(page, 0, g, slot, d)];",
                         "k_out[dst] = pool[o_offset(page, 1, g, slot, d)];"),
 }
@@ -42,6 +48,8 @@ PIN_CALLS = [
     pins.test_append_writes_exactly_one_slot_per_kv_head,
     pins.test_append_then_single_token_decode_returns_v_new,
     pins.test_gather_matches_fancy_indexing_and_leaves_tail,
+    pins.test_fill_equals_successive_appends,
+    pins.test_fill_then_gather_returns_the_tokens,
 ]
 
 
