@@ -2,14 +2,15 @@
 """Benchmark of the paged decode-attention hot path on B200.
 
 One step = one decode step of the whole model's attention cache traffic:
-for each of the 16 layers, append the new token's K/V of every sequence
-(pkv_append) and run decode attention over the paged cache
-(paged_attention_decode), through the C ABI.  Default workload: the
+for each of the 16 layers, append the new token's K/V of every sequence and
+run decode attention over the paged cache, through the C ABI -- by default
+as one fused call per layer (paged_attention_decode_append), with --unfused
+as pkv_append then paged_attention_decode.  Default workload: the
 continuous-batching mix (batch 64, lengths log-uniform in [1, 8192],
 fragmented block tables, 16 layers).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--kernel auto|simt|mma]
+                    [--impl ours|reference] [--kernel auto|simt|mma] [--unfused]
 
 Prints one JSON line (rank 0).  ``value`` is decode-queries/s over all
 ranks, one query being one sequence's 32 query heads at one layer.  The
@@ -185,12 +186,13 @@ def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
 class Runner:
     """Device-resident state of one workload on one GPU."""
 
-    def __init__(self, w: W.Workload, device, kernel: int):
+    def __init__(self, w: W.Workload, device, kernel: int, fused: bool):
         from paged_attention_decode_pkv_b200 import pkv
         self.pkv = pkv
         self.w = w
         self.device = device
         self.kernel = kernel
+        self.fused = fused
         self.pool_t = W.make_pool(w, device)
         self.pool = pkv.Pool(w.num_pages, storage=self.pool_t)
         self.bt = torch.from_numpy(w.block_tables).to(device)
@@ -207,10 +209,16 @@ class Runner:
 
     def launch_step(self, stream, variant, decode_only=False):
         """Launch one decode step (all layers) for lengths variant `variant`:
-        append + decode per layer, or only the decodes."""
+        per layer the fused append + decode, or append then decode, or (for
+        the unfused decode roofline) only the decodes."""
         pkv = self.pkv
         sl = self.seq_lens[variant]
         for l in range(self.w.num_layers):
+            if self.fused:
+                pkv.decode_append(self.q[l], self.k[l], self.v[l], self.pool, self.bt, sl, l,
+                                  self.w.scale, out=self.out[l], workspace=self.ws,
+                                  kernel=self.kernel, stream=stream)
+                continue
             if not decode_only:
                 pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
             pkv.decode(self.q[l], self.pool, self.bt, sl, l, self.w.scale, out=self.out[l],
@@ -222,8 +230,10 @@ class Runner:
         No timing events inside the graphs: an event node costs a few
         microseconds and would break the launch chaining."""
         self.graphs, self.decode_graphs = [], []
+        kinds = ((False, self.graphs),) if self.fused else \
+            ((False, self.graphs), (True, self.decode_graphs))
         for v in range(self.w.num_steps):
-            for only, dst in ((False, self.graphs), (True, self.decode_graphs)):
+            for only, dst in kinds:
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=stream):
                     self.launch_step(stream, v, decode_only=only)
@@ -236,8 +246,11 @@ class Runner:
         self.decode_graphs[i % len(self.decode_graphs)].replay()
 
     def decode_bytes(self, i):
-        """Algorithmic bytes of one decode launch of lengths variant i."""
-        return alg_bytes_decode(self.w.seq_lens(i % self.w.num_steps + 1))
+        """Algorithmic bytes of one decode launch of lengths variant i (with
+        the fused append: plus each sequence's new K/V rows read from the
+        inputs and written into the pool)."""
+        b = alg_bytes_decode(self.w.seq_lens(i % self.w.num_steps + 1))
+        return b + (4096 * self.w.batch if self.fused else 0)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -246,9 +259,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     kernel = {"auto": pkv.KERNEL_AUTO, "simt": pkv.KERNEL_SIMT, "mma": pkv.KERNEL_MMA}[args.kernel]
     w = workload_for_rank(args.workload, rank)
-    r = Runner(w, device, kernel)
+    fused = not args.unfused
+    r = Runner(w, device, kernel, fused)
     if not args.no_pdl:
-        # appends precede every decode and only read the tables
+        # no kernel of the step writes the lengths or the block tables
         r.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
@@ -261,12 +275,14 @@ def run_ours(args, rank, world, local_rank):
         r.replay(i)
     torch.cuda.synchronize()
 
-    # ---- timed region: (A) K full steps, then (B) the decodes of K steps
-    # alone, back to back, for the decode kernel's launch duration
+    # ---- timed region: (A) K full steps; unfused only, then (B) the decodes
+    # of K steps alone, back to back, for the decode kernel's launch duration
+    # (fused, a step is nothing but the decode launches, so (A) gives it)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for i in range(max(args.warmup, w.num_steps)):
-        r.replay_decodes(i)
+    if not fused:
+        for i in range(max(args.warmup, w.num_steps)):
+            r.replay_decodes(i)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
@@ -275,16 +291,18 @@ def run_ours(args, rank, world, local_rank):
             for i in range(args.steps):
                 r.replay(i)
             t1.record(stream)
-            d0.record(stream)
-            for i in range(args.steps):
-                r.replay_decodes(i)
-            d1.record(stream)
+            if not fused:
+                d0.record(stream)
+                for i in range(args.steps):
+                    r.replay_decodes(i)
+                d1.record(stream)
         stream.synchronize()
         torch.cuda.synchronize()
     barrier()
     ms = t0.elapsed_time(t1)
     dec_launches = args.steps * w.num_layers
-    avg_dec_s = max_over_ranks(d0.elapsed_time(d1), device) / dec_launches / 1e3
+    dec_ms = t0.elapsed_time(t1) if fused else d0.elapsed_time(d1)
+    avg_dec_s = max_over_ranks(dec_ms, device) / dec_launches / 1e3
     avg_bytes = sum(r.decode_bytes(i) for i in range(args.steps)) / args.steps
     err = pkv.get_device_error(r.pool, stream)
     if err != 0:
@@ -312,26 +330,32 @@ def run_ours(args, rank, world, local_rank):
             "layers": w.num_layers, "pool_pages": w.num_pages,
             "kv_bytes_per_layer": w.kv_bytes(1), "accumulate": "f32",
             "kernel": args.kernel, "parallelism": "dp%d (independent replicas)" % world,
-            "launch": "one CUDA graph per step (16 x append + decode + split merge)%s" %
-                      ("" if args.no_pdl else ", programmatic dependent launch, "
-                                             "tables read before the append ends"),
+            "launch": "one CUDA graph per step (16 x %s + split merge)%s" %
+                      ("fused append+decode" if fused else "append + decode",
+                       "" if args.no_pdl else ", programmatic dependent launch, tables read "
+                                              "before the preceding kernel ends"),
             "l2": "inputs larger than L2: one step reads %.0f MB of K/V" %
                   (w.kv_bytes(1) * w.num_layers / 1e6),
         },
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-            "kernel": "decode_kernel (+ split-KV merge_kernel)",
+            "kernel": "decode_kernel%s (+ split-KV merge_kernel)" %
+                      (" with fused append" if fused else ""),
             "alg_bytes_per_launch": avg_bytes, "avg_launch_us": avg_dec_s * 1e6,
             "launches": dec_launches,
         },
-        "decode_only_queries_per_s": w.batch / avg_dec_s,
+        "decode_queries_per_s": w.batch / avg_dec_s,
         "e2e": e2e,
         "prefill_fill": fill,
-        "gpu_launches": args.steps * w.num_layers * 3 + dec_launches * 2,
-        "decode_timing": "CUDA events around %d back-to-back replays of the step's decode "
-                         "launches alone (decode + merge per layer, %d launches)" %
-                         (args.steps, dec_launches),
+        "gpu_launches": (args.steps * w.num_layers * 2 if fused else
+                         args.steps * w.num_layers * 3 + dec_launches * 2),
+        "decode_timing": ("CUDA events around the %d full-step replays (fused append + decode "
+                          "+ merge per layer, %d launches)" % (args.steps, dec_launches)
+                          if fused else
+                          "CUDA events around %d back-to-back replays of the step's decode "
+                          "launches alone (decode + merge per layer, %d launches)" %
+                          (args.steps, dec_launches)),
         "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline:
@@ -523,6 +547,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fill", action="store_true", help="skip the prefill fill timing")
+    ap.add_argument("--unfused", action="store_true",
+                    help="separate append and decode launches instead of the fused call")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch")
     args = ap.parse_args()

@@ -252,6 +252,40 @@ PKV_API int paged_attention_decode_ex(const uint16_t *q, const pkv_pool *pool,
                               pkv_stream_t stream, int32_t kernel, int32_t grid_ctas,
                               int32_t min_chunk);
 
+/*
+ * Fused append + decode: exactly pkv_append(k_new, v_new) followed by
+ * paged_attention_decode with the same seq_lens, in one launch (plus the
+ * split-KV merge).  Decode adds the new token to the cache and attends to it
+ * (comrad404 article on samir-vllm, section "Что README говорит о KV-кэше и
+ * пакетном декодировании").  The CTA that reads sequence b's last page
+ * writes the new token's rows into slot (L-1) % 16 of that page, both in
+ * the pool and in its staged copy, so the page is read once and no append
+ * launch is needed.  k_new, v_new: dev BF16 [batch][8][64], 16-byte aligned.
+ * Differences from the two calls: a sequence with L = 0 gets no append and
+ * a zero output row without an error (an idle batch slot); the appended
+ * slot must not lie in another sequence's context in this call (a page that
+ * several sequences read is read-only).  Errors and outputs otherwise as
+ * pkv_append and paged_attention_decode; a page outside the pool is neither
+ * read nor written.  Workspace: pkv_decode_workspace_bytes[_ex].
+ */
+PKV_API int paged_attention_decode_append(const uint16_t *q, const uint16_t *k_new,
+                                          const uint16_t *v_new, pkv_pool *pool,
+                                          const int32_t *block_tables, const int32_t *seq_lens,
+                                          int32_t layer, float scale, float *out,
+                                          int32_t num_layers, int32_t batch, int32_t max_blocks,
+                                          void *workspace, size_t workspace_bytes,
+                                          pkv_stream_t stream);
+
+/* As paged_attention_decode_append, with the knobs of paged_attention_decode_ex. */
+PKV_API int paged_attention_decode_append_ex(const uint16_t *q, const uint16_t *k_new,
+                                             const uint16_t *v_new, pkv_pool *pool,
+                                             const int32_t *block_tables, const int32_t *seq_lens,
+                                             int32_t layer, float scale, float *out,
+                                             int32_t num_layers, int32_t batch, int32_t max_blocks,
+                                             void *workspace, size_t workspace_bytes,
+                                             pkv_stream_t stream, int32_t kernel,
+                                             int32_t grid_ctas, int32_t min_chunk);
+
 /* Workspace bytes for paged_attention_decode_ex with these knobs. */
 PKV_API int pkv_decode_workspace_bytes_ex(const pkv_pool *pool, int32_t batch, int32_t kernel,
                                   int32_t grid_ctas, size_t *bytes_out);

@@ -29,11 +29,19 @@
 //
 // A sequence whose pages all fall in one CTA is finished in registers.  A
 // sequence cut by range boundaries is split-KV: each piece writes (m, l, acc)
-// per kv head to the workspace and the last piece to arrive (atomic counter
-// per (sequence, kv head)) merges them in a fixed order with log-sum-exp
-// weights and writes out, so the split needs no second launch and the result
-// does not depend on which CTA finishes last.  Scores are kept in log2 units
-// (scaled by scale * log2(e)) and exponentials are exp2.
+// per kv head to the workspace, and merge_kernel, launched right after on the
+// same stream, combines the pieces in piece order with log-sum-exp weights,
+// so the result does not depend on which CTA finishes first.  Scores are kept
+// in log2 units (scaled by scale * log2(e)) and exponentials are exp2.
+//
+// Fused append (paged_attention_decode_append).  Decode attends to the token
+// that the step appends (comrad404 article on samir-vllm, section "Что README
+// говорит о KV-кэше и пакетном декодировании": decode adds the new token to
+// the cache).  With k_new / v_new given, the producer also bulk-copies the
+// new token's K and V rows (2 KiB) into the stage of the sequence's last
+// page; once the page has landed, warp g writes its head's two rows into the
+// staged page (slot (L-1) % 16) and into the pool, then computes as usual.
+// So the append costs no launch, and the page is read from HBM only once.
 //
 // Two compute variants share this skeleton:
 //  - SimtCompute: CUDA-core FP32 dot products (packed FFMA2) with
@@ -50,7 +58,11 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kWarps = kKvHeads;                    // one warp per kv head
 constexpr int kPageBytes = 2 * kKvHeads * kTileBytes;  // 32 KiB
 constexpr int kQRowsBytes = kQHeads * kRowBytes;    // a sequence's 32 query rows: 4 KiB
-constexpr int kStageBytes = kPageBytes + kQRowsBytes;
+constexpr int kNewRowsBytes = 2 * kKvHeads * kRowBytes;  // new token's K and V rows: 2 KiB
+// stage = page | query rows | new token rows; a multiple of 1024 B, so that
+// every stage keeps the 1024-B alignment the 128-byte swizzle needs
+constexpr int kStageBytes = kPageBytes + kQRowsBytes + kNewRowsBytes;
+static_assert(kStageBytes % 1024 == 0, "stage alignment");
 constexpr int kScratchBytes = 512;                  // per-warp P^T transpose buffer
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -661,7 +673,8 @@ __device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a,
 }
 
 // Producer-side description of page f (this lane's slot of a 32-page batch):
-// physical page, and (sequence << 1) | starts-a-sequence-in-this-range.
+// physical page, and (sequence << 2) | (last page of the sequence << 1) |
+// starts-a-sequence-in-this-range.
 __device__ __forceinline__ void load_page_batch(const DecodeArgs& a, const int32_t* s_pfx,
                                                 int32_t f, int32_t f_begin, int32_t f_end,
                                                 int32_t& phys, int32_t& info) {
@@ -671,7 +684,8 @@ __device__ __forceinline__ void load_page_batch(const DecodeArgs& a, const int32
     int b, j;
     locate(s_pfx, a.batch, f, b, j);
     phys = __ldg(a.bt + static_cast<int64_t>(b) * a.max_blocks + j);
-    info = (b << 1) | ((j == 0 || f == f_begin) ? 1 : 0);
+    info = (b << 2) | ((j == s_pfx[b + 1] - s_pfx[b] - 1) ? 2 : 0) |
+           ((j == 0 || f == f_begin) ? 1 : 0);
   }
 }
 
@@ -683,7 +697,8 @@ struct SmemPlan {
   static constexpr size_t full = scratch + size_t(kWarps) * kScratchBytes;
   static constexpr size_t empty = full + size_t(S) * 8;
   static constexpr size_t flags = empty + size_t(S) * 8;   // [S] bad page, [1] abort
-  static constexpr size_t tot = flags + size_t(S + 1) * 4;  // [kWarps] scan totals
+  static constexpr size_t phys = flags + size_t(S + 1) * 4;  // [S] physical page of the stage
+  static constexpr size_t tot = phys + size_t(S) * 4;        // [kWarps] scan totals
   static constexpr size_t lens = tot + size_t(kWarps) * 4;
   static size_t bytes(int32_t batch) {
     // lengths [B] and page-count prefix [B+1], plus 1024 B of alignment slack
@@ -702,6 +717,8 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = a.batch;
   volatile int32_t* s_flags = reinterpret_cast<int32_t*>(smem + L::flags);
+  volatile int32_t* s_phys = reinterpret_cast<int32_t*>(smem + L::phys);
+  const bool fused = a.k_new != nullptr;
   int32_t* s_len = reinterpret_cast<int32_t*>(smem + L::lens);
   int32_t* s_pfx = s_len + B;
   const uint32_t base = smem_addr(smem);
@@ -771,15 +788,23 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
       const uint32_t dst = base + L::stages + st * kStageBytes;
       const bool ok = static_cast<uint32_t>(phys) < static_cast<uint32_t>(a.num_pages);
       const bool start = info & 1;
+      const bool append = fused && (info & 2);
+      const int64_t seq = info >> 2;
       s_flags[st] = ok ? 0 : 1;
+      s_phys[st] = phys;
       if (!ok) record_error(a.err, kErrBadPage);
-      const uint32_t bytes = (ok ? kPageBytes : 0) + (start ? kQRowsBytes : 0);
+      const uint32_t bytes =
+          (ok ? kPageBytes : 0) + (start ? kQRowsBytes : 0) + (append ? kNewRowsBytes : 0);
       if (bytes) {
         mbar_arrive_expect_tx(bar, bytes);
         if (ok) tma_load_tile(dst, &tmap, 0, phys * kRowsPerPage, bar, policy);
-        if (start)
-          bulk_load(dst + kPageBytes, a.q + static_cast<int64_t>(info >> 1) * kQHeads * kDim,
-                    kQRowsBytes, bar);
+        if (start) bulk_load(dst + kPageBytes, a.q + seq * kQHeads * kDim, kQRowsBytes, bar);
+        if (append) {
+          const uint32_t nd = dst + kPageBytes + kQRowsBytes;
+          bulk_load(nd, a.k_new + seq * kKvHeads * kDim, kNewRowsBytes / 2, bar);
+          bulk_load(nd + kNewRowsBytes / 2, a.v_new + seq * kKvHeads * kDim, kNewRowsBytes / 2,
+                    bar);
+        }
       } else {
         mbar_arrive(bar);
       }
@@ -836,6 +861,25 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
     if (need_q) {
       cmp.begin(stage + kPageBytes + warp * (kGroup * kRowBytes), lane);
       need_q = false;
+    }
+    if (fused && j == np - 1) {
+      // the appended token: slot (Lb - 1) % 16 of this, the sequence's last
+      // page; lanes 0..7 move the K row of head `warp`, lanes 8..15 its V row
+      if (lane < 16) {
+        const int kv = lane >> 3, c = lane & 7;
+        const int slot = (Lb - 1) % kTokens;
+        const uint4 v = lds128(stage + kPageBytes + kQRowsBytes + kv * (kNewRowsBytes / 2) +
+                               warp * kRowBytes + c * 16);
+        const int row = kv * (kKvHeads * kTokens) + warp * kTokens + slot;
+        sts128(stage + swz(row, c), v);
+        if (!s_flags[st]) {
+          const int64_t prow = static_cast<int64_t>(s_phys[st]) * kRowsPerPage + row;
+          reinterpret_cast<uint4*>(a.pool)[prow * (kRowBytes / 16) + c] = v;
+        }
+        // the stage is refilled by TMA (async proxy) after this generic write
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
     }
     if (!s_flags[st]) {
       const int nvalid = min(kTokens, Lb - kTokens * j);

@@ -225,12 +225,16 @@ int pkv_decode_workspace_bytes(const pkv_pool* pool, int32_t batch, size_t* byte
   return pkv_decode_workspace_bytes_ex(pool, batch, PKV_KERNEL_AUTO, 0, bytes_out);
 }
 
-int paged_attention_decode_ex(const uint16_t* q, const pkv_pool* pool,
-                              const int32_t* block_tables, const int32_t* seq_lens, int32_t layer,
-                              float scale, float* out, int32_t num_layers, int32_t batch,
-                              int32_t max_blocks, void* workspace, size_t workspace_bytes,
-                              pkv_stream_t stream, int32_t kernel, int32_t grid_ctas,
-                              int32_t min_chunk) {
+}  // extern "C"
+
+namespace {
+
+// Decode, with the fused append when k_new / v_new are given.
+int decode_common(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                  const pkv_pool* pool, const int32_t* block_tables, const int32_t* seq_lens,
+                  int32_t layer, float scale, float* out, int32_t num_layers, int32_t batch,
+                  int32_t max_blocks, void* workspace, size_t workspace_bytes,
+                  pkv_stream_t stream, int32_t kernel, int32_t grid_ctas, int32_t min_chunk) {
   int s = check_table_args(pool, block_tables, seq_lens, layer, num_layers, batch, max_blocks);
   if (s != PKV_OK) return s;
   if (!q || !out || !aligned(q, 16) || !aligned(out, 16)) return PKV_ERR_INVALID_ARG;
@@ -254,8 +258,49 @@ int paged_attention_decode_ex(const uint16_t* q, const pkv_pool* pool,
   a.min_chunk = min_chunk;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.flags = pool->launch_flags;
+  a.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
+  a.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
+  a.pool = static_cast<__nv_bfloat16*>(pool->data);
   return from_cuda(pkv::launch_decode(plan, pool->tmap, a, pool->launch_flags,
                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attention_decode_ex(const uint16_t* q, const pkv_pool* pool,
+                              const int32_t* block_tables, const int32_t* seq_lens, int32_t layer,
+                              float scale, float* out, int32_t num_layers, int32_t batch,
+                              int32_t max_blocks, void* workspace, size_t workspace_bytes,
+                              pkv_stream_t stream, int32_t kernel, int32_t grid_ctas,
+                              int32_t min_chunk) {
+  return decode_common(q, nullptr, nullptr, pool, block_tables, seq_lens, layer, scale, out,
+                       num_layers, batch, max_blocks, workspace, workspace_bytes, stream, kernel,
+                       grid_ctas, min_chunk);
+}
+
+int paged_attention_decode_append_ex(const uint16_t* q, const uint16_t* k_new,
+                                     const uint16_t* v_new, pkv_pool* pool,
+                                     const int32_t* block_tables, const int32_t* seq_lens,
+                                     int32_t layer, float scale, float* out, int32_t num_layers,
+                                     int32_t batch, int32_t max_blocks, void* workspace,
+                                     size_t workspace_bytes, pkv_stream_t stream, int32_t kernel,
+                                     int32_t grid_ctas, int32_t min_chunk) {
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return PKV_ERR_INVALID_ARG;
+  return decode_common(q, k_new, v_new, pool, block_tables, seq_lens, layer, scale, out,
+                       num_layers, batch, max_blocks, workspace, workspace_bytes, stream, kernel,
+                       grid_ctas, min_chunk);
+}
+
+int paged_attention_decode_append(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                                  pkv_pool* pool, const int32_t* block_tables,
+                                  const int32_t* seq_lens, int32_t layer, float scale, float* out,
+                                  int32_t num_layers, int32_t batch, int32_t max_blocks,
+                                  void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+  return paged_attention_decode_append_ex(q, k_new, v_new, pool, block_tables, seq_lens, layer,
+                                          scale, out, num_layers, batch, max_blocks, workspace,
+                                          workspace_bytes, stream, PKV_KERNEL_AUTO, 0, 0);
 }
 
 int paged_attention_decode(const uint16_t* q, const pkv_pool* pool, const int32_t* block_tables,

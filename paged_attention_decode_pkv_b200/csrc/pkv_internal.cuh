@@ -169,6 +169,18 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (TMA / bulk copy) accesses to shared memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Byte offset of 16-byte chunk `c` of row `r` inside a TMA tile written with
 // the 128-byte swizzle (rows of 128 B; chunk index XOR row % 8).
 __device__ __forceinline__ uint32_t swz(int r, int c) {
@@ -204,6 +216,11 @@ struct DecodeArgs {
   int32_t min_chunk;        // minimum pages per CTA range
   float scale_log2;         // scale * log2(e)
   int32_t flags;            // kLaunch* bits
+  // Fused append (paged_attention_decode_append): the new token's K/V rows
+  // [B][8][64] and the page storage they are written into; null otherwise.
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* pool;
 };
 
 // Launch planning shared by the workspace query and the launch.

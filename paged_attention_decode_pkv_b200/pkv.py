@@ -46,7 +46,8 @@ EXPORTS = (
     "paged_attention_decode_ex", "pkv_gather", "pkv_get_device_error", "pkv_status_string",
     "pkv_last_error_message", "pkv_pool_set_launch_flags", "paged_attention_decode_noalloc",
     "pkv_fill", "pkv_allocator_create", "pkv_allocator_destroy", "pkv_allocator_free_count",
-    "pkv_allocator_alloc", "pkv_allocator_free",
+    "pkv_allocator_alloc", "pkv_allocator_free", "paged_attention_decode_append",
+    "paged_attention_decode_append_ex",
 )
 
 
@@ -76,6 +77,10 @@ def _load():
         "paged_attention_decode_noalloc": ([P, P, P, P, i32, ctypes.c_float, P, i32, i32, i32, P],
                                            ctypes.c_int),
         "pkv_fill": ([P, P, P, P, P, P, i32, i32, i32, i32, i32, P], ctypes.c_int),
+        "paged_attention_decode_append": ([P, P, P, P, P, P, i32, ctypes.c_float, P, i32, i32,
+                                           i32, P, sz, P], ctypes.c_int),
+        "paged_attention_decode_append_ex": ([P, P, P, P, P, P, i32, ctypes.c_float, P, i32, i32,
+                                              i32, P, sz, P, i32, i32, i32], ctypes.c_int),
         "pkv_allocator_create": ([i32, ctypes.POINTER(P)], ctypes.c_int),
         "pkv_allocator_destroy": ([P], ctypes.c_int),
         "pkv_allocator_free_count": ([P], i32),
@@ -226,6 +231,30 @@ def decode(q: torch.Tensor, pool: Pool, block_tables: torch.Tensor, seq_lens: to
         _dev(out, torch.float32, (B, NUM_Q_HEADS, HEAD_DIM), "out"), L, B, MB,
         _dev(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream),
         int(kernel), int(grid_ctas), int(min_chunk)), "paged_attention_decode")
+    return out
+
+
+def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, pool: Pool,
+                  block_tables: torch.Tensor, seq_lens: torch.Tensor, layer: int, scale: float,
+                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  kernel: int = KERNEL_AUTO, grid_ctas: int = 0, min_chunk: int = 0,
+                  stream=None) -> torch.Tensor:
+    """append(k_new, v_new) then decode, fused into one launch
+    (paged_attention_decode_append_ex)."""
+    L, B, MB = block_tables.shape
+    if out is None:
+        out = torch.empty((B, NUM_Q_HEADS, HEAD_DIM), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = pool.workspace(B, kernel, grid_ctas)
+    _check(lib.paged_attention_decode_append_ex(
+        _dev(q, torch.bfloat16, (B, NUM_Q_HEADS, HEAD_DIM), "q"),
+        _dev(k_new, torch.bfloat16, (B, NUM_KV_HEADS, HEAD_DIM), "k_new"),
+        _dev(v_new, torch.bfloat16, (B, NUM_KV_HEADS, HEAD_DIM), "v_new"), pool.handle,
+        _dev(block_tables, torch.int32, None, "block_tables"),
+        _dev(seq_lens, torch.int32, (B,), "seq_lens"), int(layer), float(scale),
+        _dev(out, torch.float32, (B, NUM_Q_HEADS, HEAD_DIM), "out"), L, B, MB,
+        _dev(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream),
+        int(kernel), int(grid_ctas), int(min_chunk)), "paged_attention_decode_append")
     return out
 
 
