@@ -127,3 +127,26 @@ def decode(q, pool, block_tables, seq_lens, layer, scale, rows=None, nthreads=No
     _check(_lib().pkvo_decode(_p(q), _p(pool), pool.shape[0], _p(bt), L, B, MB, _p(sl),
                               int(layer), float(scale), _p(out), rp, nr, int(nthreads)))
     return out
+
+
+def decode_multi(q, pool, block_tables, seq_lens, layer, scale, nthreads=None):
+    """FP64 decode of several queries per sequence, causal among them.
+
+    q: uint16 [batch, T, 32, 64].  Query i of sequence b sees the tokens
+    t < seq_lens[b] - T + 1 + i (query T-1 sees the whole context, each
+    earlier query one token fewer), so its output is single-query decode at
+    that shorter length -- which is how it is computed here, one decode()
+    call per query.  A sequence with 0 < seq_lens[b] < T has a query with no
+    token: OracleError (bad length).  Returns float64 [batch, T, 32, 64].
+    """
+    q = np.asarray(q, np.uint16)
+    B, T = q.shape[0], q.shape[1]
+    sl = np.asarray(seq_lens, np.int64)
+    if ((sl > 0) & (sl < T)).any():
+        raise OracleError(2)
+    out = np.zeros((B, T, 32, 64), np.float64)
+    for i in range(T):
+        li = np.where(sl > 0, sl - T + 1 + i, 0).astype(np.int32)
+        out[:, i] = decode(np.ascontiguousarray(q[:, i]), pool, block_tables, li, layer, scale,
+                           nthreads=nthreads)
+    return out

@@ -304,3 +304,54 @@ def test_fill_rejects_out_of_range_without_writing():
     with pytest.raises(oracle.OracleError):
         oracle.fill(pool, c["bt"], cu, st, k, v, 0)
     assert np.array_equal(pool, c["pool"])
+
+
+# ---- several queries per sequence, causal among them (oracle.decode_multi)
+
+def _brute_multi(c, q2, scale=0.125):
+    """Causal two-query attention written out with an explicit mask: query i
+    of a length-L sequence scores every token and masks t > L - 2 + i."""
+    B, Tq = q2.shape[0], q2.shape[1]
+    out = np.zeros((B, Tq, H, D))
+    for b, (K, V) in enumerate(contiguous_kv(c)):
+        L = K.shape[1]
+        if L == 0:
+            continue
+        Kh = np.repeat(K, H // G, axis=0)
+        Vh = np.repeat(V, H // G, axis=0)
+        for i in range(Tq):
+            q = bf16_to_f64(q2[b, i])
+            s = scale * np.einsum("hd,hld->hl", q, Kh)
+            s[:, np.arange(L) > L - Tq + i] = -np.inf
+            s -= s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, i] = np.einsum("hl,hld->hd", p, Vh)
+    return out
+
+
+@pytest.mark.parametrize("lens", [[2], [16], [17], [18], [33, 2, 0, 40]])
+def test_decode_multi_matches_causal_bruteforce(lens):
+    c = make_case(lens, seed=sum(lens) + 3)
+    rng = np.random.default_rng(len(lens))
+    q2 = bf16_bits(rng.standard_normal((len(lens), 2, H, D)))
+    got = oracle.decode_multi(q2, c["pool"], c["bt"], c["seq_lens"], 0, 0.125)
+    assert np.max(np.abs(got - _brute_multi(c, q2))) <= 1e-12
+
+
+def test_decode_multi_one_query_is_decode_and_last_query_sees_all():
+    c = make_case([40, 2, 17], seed=21)
+    got1 = oracle.decode_multi(c["q"][:, None], c["pool"], c["bt"], c["seq_lens"], 0, 0.2)
+    assert np.array_equal(got1[:, 0], _decode(c, scale=0.2))
+    rng = np.random.default_rng(4)
+    q2 = bf16_bits(rng.standard_normal((3, 2, H, D)))
+    q2[:, 1] = c["q"]
+    got2 = oracle.decode_multi(q2, c["pool"], c["bt"], c["seq_lens"], 0, 0.2)
+    assert np.array_equal(got2[:, 1], _decode(c, scale=0.2))   # the last query: plain decode
+
+
+def test_decode_multi_rejects_a_query_without_tokens():
+    c = make_case([1, 5], seed=2)
+    with pytest.raises(oracle.OracleError):
+        oracle.decode_multi(np.zeros((2, 2, H, D), np.uint16), c["pool"], c["bt"],
+                            c["seq_lens"], 0, 0.125)
