@@ -44,12 +44,14 @@ FALLBACK_HBM_GBS = 6650.0
 
 # ------------------------------------------------------------------ helpers --
 
-def alg_bytes_decode(seq_lens: np.ndarray) -> int:
+def alg_bytes_decode(seq_lens: np.ndarray, queries: int = 1, out_bytes: int = 4) -> int:
     """Algorithmic bytes of one decode launch: per sequence K+V of every
-    token (2048 B/token), q (4096 B), FP32 out (8192 B), block-table entries
-    (4 B per page) and the length (4 B)."""
+    token (2048 B/token), q (4096 B per query), out (32 x 64 elements of
+    out_bytes per query: 8192 B in FP32), block-table entries (4 B per page)
+    and the length (4 B)."""
     L = seq_lens.astype(np.int64)
-    return int((2048 * L + 4096 + 8192 + 4 * ((L + 15) // 16) + 4).sum())
+    per_seq = 2048 * L + queries * (4096 + 2048 * out_bytes) + 4 * ((L + 15) // 16) + 4
+    return int(per_seq.sum())
 
 
 def kernel_source_digest() -> str:
@@ -186,26 +188,38 @@ def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
 class Runner:
     """Device-resident state of one workload on one GPU."""
 
-    def __init__(self, w: W.Workload, device, kernel: int, fused: bool):
+    def __init__(self, w: W.Workload, device, kernel: int, fused: bool, queries: int = 1,
+                 out_dtype=torch.float32):
         from paged_attention_decode_pkv_b200 import pkv
         self.pkv = pkv
         self.w = w
         self.device = device
         self.kernel = kernel
-        self.fused = fused
-        self.pool_t = W.make_pool(w, device)
+        self.queries = queries
+        self.out_dtype = out_dtype
+        # two queries per sequence: decode only (their tokens would be
+        # written with pkv_fill, not the one-token fused append)
+        self.fused = fused and queries == 1
+        # Two queries need a context of at least two tokens: such sequences get
+        # length max(L, 2), and the pool holds values (not NaN) in every slot,
+        # the second token of a one-token sequence included.
+        self.pool_t = W.make_pool(w, device, poison=queries == 1)
         self.pool = pkv.Pool(w.num_pages, storage=self.pool_t)
         self.bt = torch.from_numpy(w.block_tables).to(device)
         nl, B = w.num_layers, w.batch
-        self.seq_lens = [torch.from_numpy(w.seq_lens(s)).to(device)
-                         for s in range(1, w.num_steps + 1)]
+        self.lens_np = [np.maximum(w.seq_lens(s), queries).astype(np.int32)
+                        for s in range(1, w.num_steps + 1)]
+        self.seq_lens = [torch.from_numpy(x).to(device) for x in self.lens_np]
         # one set of per-layer inputs, reused every step (values do not change timing)
         ins = [W.step_inputs(w, 1, l, device) for l in range(nl)]
         self.q = torch.stack([x[0] for x in ins])
+        if queries == 2:   # a second query per sequence: the first one again, shifted in value
+            self.q = torch.stack([self.q, (self.q.float() * 0.5).to(torch.bfloat16)], dim=2)
         self.k = torch.stack([x[1] for x in ins])
         self.v = torch.stack([x[2] for x in ins])
-        self.out = torch.empty((nl, B, 32, 64), dtype=torch.float32, device=device)
-        self.ws = self.pool.workspace(B, kernel)
+        oshape = (nl, B, 32, 64) if queries == 1 else (nl, B, queries, 32, 64)
+        self.out = torch.empty(oshape, dtype=out_dtype, device=device)
+        self.ws = self.pool.workspace(B, kernel, 0, queries)
 
     def launch_step(self, stream, variant, decode_only=False):
         """Launch one decode step (all layers) for lengths variant `variant`:
@@ -214,6 +228,15 @@ class Runner:
         pkv = self.pkv
         sl = self.seq_lens[variant]
         for l in range(self.w.num_layers):
+            if self.queries == 2 or self.out_dtype != torch.float32:
+                kv = dict(k_new=self.k[l], v_new=self.v[l]) if self.fused else {}
+                if not self.fused and not decode_only and self.queries == 1:
+                    pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
+                pkv.decode_general(self.q[l], self.pool, self.bt, sl, l, self.w.scale,
+                                   num_queries=self.queries, out_dtype=self.out_dtype,
+                                   out=self.out[l], workspace=self.ws, kernel=self.kernel,
+                                   stream=stream, **kv)
+                continue
             if self.fused:
                 pkv.decode_append(self.q[l], self.k[l], self.v[l], self.pool, self.bt, sl, l,
                                   self.w.scale, out=self.out[l], workspace=self.ws,
@@ -249,7 +272,8 @@ class Runner:
         """Algorithmic bytes of one decode launch of lengths variant i (with
         the fused append: plus each sequence's new K/V rows read from the
         inputs and written into the pool)."""
-        b = alg_bytes_decode(self.w.seq_lens(i % self.w.num_steps + 1))
+        b = alg_bytes_decode(self.lens_np[i % self.w.num_steps], self.queries,
+                             self.out.element_size())
         return b + (4096 * self.w.batch if self.fused else 0)
 
 
@@ -259,8 +283,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     kernel = {"auto": pkv.KERNEL_AUTO, "simt": pkv.KERNEL_SIMT, "mma": pkv.KERNEL_MMA}[args.kernel]
     w = workload_for_rank(args.workload, rank)
-    fused = not args.unfused
-    r = Runner(w, device, kernel, fused)
+    fused = not args.unfused and args.queries == 1
+    out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+    r = Runner(w, device, kernel, fused, args.queries, out_dtype)
     if not args.no_pdl:
         # no kernel of the step writes the lengths or the block tables
         r.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES)
@@ -308,7 +333,7 @@ def run_ours(args, rank, world, local_rank):
     if err != 0:
         raise RuntimeError("device error during timed region: %s" % pkv.status_string(err))
     ms = max_over_ranks(ms, device)
-    value = whole_job_rate(args.steps * w.num_layers * w.batch, world, ms)
+    value = whole_job_rate(args.steps * w.num_layers * w.batch * r.queries, world, ms)
 
     # ---- end to end through the public API from pinned host buffers
     e2e = run_e2e(r, stream, min(args.steps, args.e2e_steps), device, world)
@@ -330,8 +355,10 @@ def run_ours(args, rank, world, local_rank):
             "layers": w.num_layers, "pool_pages": w.num_pages,
             "kv_bytes_per_layer": w.kv_bytes(1), "accumulate": "f32",
             "kernel": args.kernel, "parallelism": "dp%d (independent replicas)" % world,
+            "queries_per_sequence": r.queries, "out_dtype": args.out_dtype,
             "launch": "one CUDA graph per step (16 x %s + split merge)%s" %
-                      ("fused append+decode" if fused else "append + decode",
+                      ("fused append+decode" if fused else
+                       "two-query decode" if r.queries == 2 else "append + decode",
                        "" if args.no_pdl else ", programmatic dependent launch, tables read "
                                               "before the preceding kernel ends"),
             "l2": "inputs larger than L2: one step reads %.0f MB of K/V" %
@@ -345,11 +372,11 @@ def run_ours(args, rank, world, local_rank):
             "alg_bytes_per_launch": avg_bytes, "avg_launch_us": avg_dec_s * 1e6,
             "launches": dec_launches,
         },
-        "decode_queries_per_s": w.batch / avg_dec_s,
+        "decode_queries_per_s": w.batch * r.queries / avg_dec_s,
         "e2e": e2e,
         "prefill_fill": fill,
-        "gpu_launches": (args.steps * w.num_layers * 2 if fused else
-                         args.steps * w.num_layers * 3 + dec_launches * 2),
+        "gpu_launches": (args.steps * w.num_layers * (2 if fused or r.queries == 2 else 3) +
+                         (0 if fused else dec_launches * 2)),
         "decode_timing": ("CUDA events around the %d full-step replays (fused append + decode "
                           "+ merge per layer, %d launches)" % (args.steps, dec_launches)
                           if fused else
@@ -392,7 +419,8 @@ def run_e2e(r: Runner, stream, steps, device, world):
     stream.synchronize()
     barrier()
     ms = max_over_ranks(t0.elapsed_time(t1), device)
-    return {"value": whole_job_rate(steps * w.num_layers * w.batch, world, ms), "unit": UNIT,
+    return {"value": whole_job_rate(steps * w.num_layers * w.batch * r.queries, world, ms),
+            "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps}
 
@@ -547,6 +575,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fill", action="store_true", help="skip the prefill fill timing")
+    ap.add_argument("--queries", type=int, default=1, choices=[1, 2],
+                    help="queries per sequence (2: causal pair, decode only)")
+    ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])
     ap.add_argument("--unfused", action="store_true",
                     help="separate append and decode launches instead of the fused call")
     ap.add_argument("--no-pdl", action="store_true",

@@ -286,6 +286,64 @@ PKV_API int paged_attention_decode_append_ex(const uint16_t *q, const uint16_t *
                                              pkv_stream_t stream, int32_t kernel,
                                              int32_t grid_ctas, int32_t min_chunk);
 
+/*
+ * General decode call: every option of the calls above, plus two that they
+ * lack, in one parameter block (future fields are appended; struct_size
+ * tells the library which fields the caller knows).
+ *
+ *  - num_queries = 2: two queries per sequence, causal between them (the
+ *    plainest multi-token decode, as in checking a drafted token): q and out
+ *    are [batch][2][32][64]; query i of sequence b attends to tokens
+ *    t < seq_lens[b] - 1 + i, i.e. query 0 does not see the last token.
+ *    Needs seq_lens[b] = 0 or >= 2 (1 -> PKV_ERR_BAD_SEQ_LEN, zero rows),
+ *    the tensor-core kernel (PKV_KERNEL_SIMT -> PKV_ERR_UNSUPPORTED) and no
+ *    fused append (k_new must be NULL: write the two tokens with pkv_fill).
+ *  - out_dtype = PKV_DTYPE_BF16: the output rows are BF16, rounded to
+ *    nearest even from the FP32 result (the pages warn that BF16 rounding
+ *    can differ with the batch size: "Curso gratuito recorre la inferencia
+ *    de LLM...", the note on batch-dependent BF16 rounding).
+ *
+ * Fields: q (dev BF16 [batch][num_queries][32][64]); k_new, v_new (NULL, or
+ * dev BF16 [batch][8][64]: fused append as paged_attention_decode_append);
+ * block_tables, seq_lens, layer, num_layers, batch, max_blocks, scale as in
+ * paged_attention_decode; out (dev [batch][num_queries][32][64] of
+ * out_dtype, 16-byte aligned); workspace, workspace_bytes (see
+ * pkv_decode_params_workspace_bytes); kernel, grid_ctas, min_chunk as in
+ * paged_attention_decode_ex.  Errors as paged_attention_decode.
+ */
+#define PKV_DTYPE_F32 0
+#define PKV_DTYPE_BF16 1
+
+typedef struct pkv_decode_params {
+  size_t struct_size; /* sizeof(pkv_decode_params) */
+  const uint16_t *q;
+  const uint16_t *k_new;
+  const uint16_t *v_new;
+  const int32_t *block_tables;
+  const int32_t *seq_lens;
+  void *out;
+  void *workspace;
+  size_t workspace_bytes;
+  float scale;
+  int32_t layer;
+  int32_t num_layers;
+  int32_t batch;
+  int32_t max_blocks;
+  int32_t num_queries; /* 1 or 2 */
+  int32_t out_dtype;   /* PKV_DTYPE_F32 or PKV_DTYPE_BF16 */
+  int32_t kernel;
+  int32_t grid_ctas;
+  int32_t min_chunk;
+} pkv_decode_params;
+
+PKV_API int pkv_decode(pkv_pool *pool, const pkv_decode_params *params, pkv_stream_t stream);
+
+/* Workspace bytes pkv_decode needs for these parameters (only batch,
+ * num_queries, kernel and grid_ctas are read). */
+PKV_API int pkv_decode_params_workspace_bytes(const pkv_pool *pool,
+                                              const pkv_decode_params *params,
+                                              size_t *bytes_out);
+
 /* Workspace bytes for paged_attention_decode_ex with these knobs. */
 PKV_API int pkv_decode_workspace_bytes_ex(const pkv_pool *pool, int32_t batch, int32_t kernel,
                                   int32_t grid_ctas, size_t *bytes_out);

@@ -46,10 +46,12 @@
 // Two compute variants share this skeleton:
 //  - SimtCompute: CUDA-core FP32 dot products (packed FFMA2) with
 //    warp-shuffle reductions for the dot products, the max and the sum;
-//  - MmaCompute: the 16-token x 4-head tile on the tensor cores
+//  - MmaComputeT<n>: the 16-token x 4-head tile on the tensor cores
 //    (mma.sync m16n8k16, BF16 in, FP32 accumulate) for both Q.K^T and P.V,
 //    with P split into two BF16 terms (hi + lo) so that rounding P to BF16
-//    costs no accuracy; softmax stays FP32 on the CUDA cores.
+//    costs no accuracy; softmax stays FP32 on the CUDA cores.  The MMA's
+//    N = 8 holds 4 heads; with n = 2 the other 4 columns carry a second query
+//    of the same sequence (causal: it sees one token more than the first).
 #include "pkv_internal.cuh"
 
 namespace pkv {
@@ -57,12 +59,17 @@ namespace pkv {
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kWarps = kKvHeads;                    // one warp per kv head
 constexpr int kPageBytes = 2 * kKvHeads * kTileBytes;  // 32 KiB
-constexpr int kQRowsBytes = kQHeads * kRowBytes;    // a sequence's 32 query rows: 4 KiB
+constexpr int kQRowsBytes = kQHeads * kRowBytes;    // one query's 32 head rows: 4 KiB
 constexpr int kNewRowsBytes = 2 * kKvHeads * kRowBytes;  // new token's K and V rows: 2 KiB
-// stage = page | query rows | new token rows; a multiple of 1024 B, so that
-// every stage keeps the 1024-B alignment the 128-byte swizzle needs
-constexpr int kStageBytes = kPageBytes + kQRowsBytes + kNewRowsBytes;
-static_assert(kStageBytes % 1024 == 0, "stage alignment");
+// stage = page | query rows (nq queries) | new token rows; a multiple of
+// 1024 B, so that every stage keeps the 1024-B alignment the 128-byte
+// swizzle needs
+template <int nq>
+struct StageLayout {
+  static constexpr int kQBytes = nq * kQRowsBytes;
+  static constexpr int kBytes = kPageBytes + kQBytes + kNewRowsBytes;
+  static_assert(kBytes % 1024 == 0, "stage alignment");
+};
 constexpr int kScratchBytes = 512;                  // per-warp P^T transpose buffer
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -70,6 +77,45 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// Output rows of one (sequence, kv head) unit: element (query i, head h of
+// the group, dim d) is at base + i * qstride + h * 64 + d, FP32 or BF16
+// (rounded to nearest even).  Partial records use the same shape in FP32.
+struct OutRows {
+  void* base;
+  int64_t qstride;   // elements
+  bool bf16;
+
+  __device__ __forceinline__ int64_t at(int i, int h, int d) const {
+    return i * qstride + h * kDim + d;
+  }
+  __device__ __forceinline__ void put(int i, int h, int d, float v) const {
+    if (bf16)
+      static_cast<__nv_bfloat16*>(base)[at(i, h, d)] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(base)[at(i, h, d)] = v;
+  }
+  // dims d, d + 1 (d even)
+  __device__ __forceinline__ void put2(int i, int h, int d, float x, float y) const {
+    if (bf16)
+      *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(base) + at(i, h, d)) =
+          pack_bf16x2(x, y);
+    else
+      *reinterpret_cast<float2*>(static_cast<float*>(base) + at(i, h, d)) = make_float2(x, y);
+  }
+  // dims d .. d + 7 (d a multiple of 8)
+  __device__ __forceinline__ void put8(int i, int h, int d, const float* v) const {
+    if (bf16) {
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + at(i, h, d)) =
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                     pack_bf16x2(v[6], v[7]));
+    } else {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(base) + at(i, h, d));
+      dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+      dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+};
 
 // ---------------------------------------------------------------------------
 // CUDA-core compute: FP32 dot products with packed FFMA2, warp-shuffle
@@ -87,13 +133,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
 struct SimtCompute {
   static constexpr int kStages = 3;
   static constexpr int kMinBlocks = 1;
+  static constexpr int kQueries = 1;
 
   float2 q2[kGroup][4];   // q[h][8c + 2e], q[h][8c + 2e + 1]
   float2 acc[kGroup][4];  // sum over this lane's tokens of p * v[8c + 2e ..]
   float m[kGroup];        // running max per head (log2 units), warp-uniform
   float lsum[2];          // sum of p over this lane's scores, heads 2*b2 + k
 
-  __device__ __forceinline__ void begin(uint32_t qslot, int lane) {
+  // (one query per sequence: the CUDA-core variant does not take two)
+  __device__ __forceinline__ void begin(uint32_t qrows, int warp, int /*nq*/, int lane) {
+    const uint32_t qslot = qrows + warp * (kGroup * kRowBytes);
     const int c = lane & 7;
 #pragma unroll
     for (int h = 0; h < kGroup; ++h) {
@@ -110,7 +159,8 @@ struct SimtCompute {
   }
 
   __device__ __forceinline__ void consume(uint32_t ktile, uint32_t vtile, uint32_t /*scratch*/,
-                                          int nvalid, float scale_log2, int lane) {
+                                          int nvalid, int /*nvalid_q0*/, float scale_log2,
+                                          int lane) {
     const int c = lane & 7, tg = lane >> 3;
     const int b0 = c & 1, b1 = (c >> 1) & 1, b2 = c >> 2;
 
@@ -255,19 +305,19 @@ struct SimtCompute {
     l[3] = b2 ? s2[1] : o1;
   }
 
-  __device__ __forceinline__ void finalize(float* out_rows, int lane) const {
+  __device__ __forceinline__ void finalize(const OutRows& out, int /*nq*/, int lane) const {
     float r[8], l[4];
     const int h = reduce_acc(r, lane);
     reduce_l(l, lane);
     const float lh = h == 0 ? l[0] : h == 1 ? l[1] : h == 2 ? l[2] : l[3];
     const float inv = 1.f / lh;
-    float4* dst = reinterpret_cast<float4*>(out_rows + h * kDim + 8 * (lane & 7));
-    dst[0] = make_float4(r[0] * inv, r[1] * inv, r[2] * inv, r[3] * inv);
-    dst[1] = make_float4(r[4] * inv, r[5] * inv, r[6] * inv, r[7] * inv);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) r[k] *= inv;
+    out.put8(0, h, 8 * (lane & 7), r);
   }
 
   // Partial record: m[4], l[4], acc[4][64] (unnormalised).
-  __device__ __forceinline__ void store_partial(float* P, int lane) const {
+  __device__ __forceinline__ void store_partial(float* P, int /*nq*/, int lane) const {
     float r[8], l[4];
     const int h = reduce_acc(r, lane);
     reduce_l(l, lane);
@@ -300,21 +350,29 @@ struct SimtCompute {
 //  Lane holds O^T[16mt + r (+8)][2qd..2qd+1]: its softmax heads and its
 //  accumulator heads are the same, so rescaling needs no data movement.
 // ---------------------------------------------------------------------------
-struct MmaCompute {
+template <int kNq>   // queries per sequence: 1, or 2 in the zero columns
+struct MmaComputeT {
   static constexpr int kStages = 2;
   static constexpr int kMinBlocks = 2;
+  static constexpr int kQueries = kNq;
 
   uint32_t qb[4][2];  // B fragments of Q^T, k-steps 0..3 (zero for lanes with r >= 4)
   float o[4][4];      // O^T accumulators, m-tiles 0..3
   float m[2];         // running max of heads 2qd, 2qd+1 (log2 units)
   float l[2];         // this lane's share of the softmax denominators
 
-  __device__ __forceinline__ void begin(uint32_t qslot, int lane) {
+  // qrows: the staged query rows ([query][32 heads][64]); column n of the
+  // MMA's N = 8 is head n % 4 of query n / 4 (the columns of a second query
+  // stay zero when there is one).
+  __device__ __forceinline__ void begin(uint32_t qrows, int warp, int /*nq*/, int lane) {
     const int r = lane >> 2, qd = lane & 3;
+    const int qi = r / kGroup;
+    constexpr int nq = kNq;
+    const uint32_t row = qrows + (qi * kQHeads + warp * kGroup + r % kGroup) * kRowBytes;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      if (r < kGroup) {
-        const uint32_t a = qslot + r * kRowBytes + (16 * ks + 2 * qd) * 2;
+      if (qi < nq) {
+        const uint32_t a = row + (16 * ks + 2 * qd) * 2;
         qb[ks][0] = lds32(a);
         qb[ks][1] = lds32(a + 16);
       } else {
@@ -329,8 +387,10 @@ struct MmaCompute {
     l[0] = l[1] = 0.f;
   }
 
+  // nvalid: tokens of this page in the context of the last query; nvalid_q0:
+  // in the context of query 0 of two (one fewer at the end; may be 0).
   __device__ __forceinline__ void consume(uint32_t ktile, uint32_t vtile, uint32_t scratch,
-                                          int nvalid, float scale_log2, int lane) {
+                                          int nvalid, int nvalid_q0, float scale_log2, int lane) {
     const int r = lane >> 2, qd = lane & 3;
     // ---- S^T = K Q^T
     float s[4] = {0.f, 0.f, 0.f, 0.f};
@@ -340,8 +400,10 @@ struct MmaCompute {
       ldsm_x4(a, ktile + swz(lane & 15, 2 * ks + (lane >> 4)));
       mma_bf16_16816(s, a, qb[ks][0], qb[ks][1]);
     }
-    // ---- FP32 online softmax; tokens r and r + 8, heads 2qd and 2qd + 1
-    const bool v0 = r < nvalid, v1 = r + 8 < nvalid;
+    // ---- FP32 online softmax; tokens r and r + 8, columns 2qd and 2qd + 1
+    // (query qd / 2)
+    const int nv = (kNq == 2 && qd < 2) ? nvalid_q0 : nvalid;
+    const bool v0 = r < nv, v1 = r + 8 < nv;
     const float x0 = v0 ? s[0] * scale_log2 : -INFINITY;
     const float x1 = v0 ? s[1] * scale_log2 : -INFINITY;
     const float x2 = v1 ? s[2] * scale_log2 : -INFINITY;
@@ -353,11 +415,16 @@ struct MmaCompute {
       mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
     }
     const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-    const float a0 = fast_exp2(m[0] - mn0), a1 = fast_exp2(m[1] - mn1);
+    // a column with no valid score yet (query 0's context can end a page
+    // early) keeps m = -inf: subtract 0 there, so that -inf - -inf never
+    // appears; its p and the rescale factor are then 0
+    const float r0 = (kNq == 2 && mn0 == -INFINITY) ? 0.f : mn0;
+    const float r1 = (kNq == 2 && mn1 == -INFINITY) ? 0.f : mn1;
+    const float a0 = fast_exp2(m[0] - r0), a1 = fast_exp2(m[1] - r1);
     m[0] = mn0;
     m[1] = mn1;
-    const float p0 = fast_exp2(x0 - mn0), p1 = fast_exp2(x1 - mn1);
-    const float p2 = fast_exp2(x2 - mn0), p3 = fast_exp2(x3 - mn1);
+    const float p0 = fast_exp2(x0 - r0), p1 = fast_exp2(x1 - r1);
+    const float p2 = fast_exp2(x2 - r0), p3 = fast_exp2(x3 - r1);
     l[0] = fmaf(l[0], a0, p0 + p2);
     l[1] = fmaf(l[1], a1, p1 + p3);
     // ---- P^T, split into BF16 hi + lo, through the scratch ([t][8 heads])
@@ -412,41 +479,47 @@ struct MmaCompute {
     }
   }
 
-  __device__ __forceinline__ void write_rows(float* rows, int lane, float s0, float s1) const {
+  // O^T columns 2qd, 2qd + 1 = query qd / 2, heads 2(qd % 2), 2(qd % 2) + 1,
+  // scaled by s0, s1; lanes whose query does not exist write nothing.
+  __device__ __forceinline__ void write_rows(const OutRows& out, int /*nq*/, int lane, float s0,
+                                             float s1) const {
+    constexpr int nq = kNq;
     const int r = lane >> 2, qd = lane & 3;
-    if (qd < 2) {
-      float* h0 = rows + (2 * qd) * kDim + r;
-      float* h1 = h0 + kDim;
+    const int qi = qd >> 1, h = 2 * (qd & 1);
+    if (qi < nq) {
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
-        h0[16 * mt] = o[mt][0] * s0;
-        h1[16 * mt] = o[mt][1] * s1;
-        h0[16 * mt + 8] = o[mt][2] * s0;
-        h1[16 * mt + 8] = o[mt][3] * s1;
+        out.put(qi, h, 16 * mt + r, o[mt][0] * s0);
+        out.put(qi, h + 1, 16 * mt + r, o[mt][1] * s1);
+        out.put(qi, h, 16 * mt + r + 8, o[mt][2] * s0);
+        out.put(qi, h + 1, 16 * mt + r + 8, o[mt][3] * s1);
       }
     }
   }
 
-  __device__ __forceinline__ void finalize(float* out_rows, int lane) const {
+  __device__ __forceinline__ void finalize(const OutRows& out, int nq, int lane) const {
     float l0, l1;
     reduce_l(l0, l1);
-    write_rows(out_rows, lane, 1.f / l0, 1.f / l1);
+    write_rows(out, nq, lane, 1.f / l0, 1.f / l1);
   }
 
-  __device__ __forceinline__ void store_partial(float* P, int lane) const {
+  // Partial records, one per query: P + i * kPartialFloats = m[4], l[4],
+  // acc[4][64] of query i (unnormalised).
+  __device__ __forceinline__ void store_partial(float* P, int /*nq*/, int lane) const {
+    constexpr int nq = kNq;
     float l0, l1;
     reduce_l(l0, l1);
-    const int qd = lane & 3;
-    if (lane < 2) {   // r == 0, qd == lane
-      P[2 * qd] = m[0];
-      P[2 * qd + 1] = m[1];
-      P[kGroup + 2 * qd] = l0;
-      P[kGroup + 2 * qd + 1] = l1;
+    const int qd = lane & 3, qi = qd >> 1, h = 2 * (qd & 1);
+    if (lane < 4 && qi < nq) {   // r == 0
+      float* rec = P + qi * kPartialFloats;
+      rec[h] = m[0];
+      rec[h + 1] = m[1];
+      rec[kGroup + h] = l0;
+      rec[kGroup + h + 1] = l1;
     }
-    write_rows(P + 2 * kGroup, lane, 1.f, 1.f);
+    write_rows(OutRows{P + 2 * kGroup, kPartialFloats, false}, nq, lane, 1.f, 1.f);
   }
 };
-
 
 // ---------------------------------------------------------------------------
 // Shared pieces of the persistent kernel
@@ -464,7 +537,7 @@ __device__ __forceinline__ void cta_lengths(const DecodeArgs& a, int32_t* s_len,
   int sum = 0;
   for (int b = b0; b < b1; ++b) {
     int L = a.seq_lens[b];
-    if (L < 0 || L > cap) {
+    if (L < 0 || L > cap || (L > 0 && L < a.num_queries)) {   // every query needs a token
       if (blockIdx.x == 0) record_error(a.err, kErrBadLen);
       L = 0;
     }
@@ -518,18 +591,29 @@ __device__ __forceinline__ void locate(const int32_t* s_pfx, int B, int32_t f, i
   j = f - s_pfx[b];
 }
 
-__device__ __forceinline__ void zero_rows(float* rows, int lane) {
-  float4* d = reinterpret_cast<float4*>(rows);
+// Zero the output rows of sequence b (all its queries), one warp.
+__device__ __forceinline__ void zero_rows(const DecodeArgs& a, int b, int lane) {
+  const int64_t bytes =
+      static_cast<int64_t>(a.num_queries) * kQHeads * kDim * (a.out_bf16 ? 2 : 4);
+  float4* d = reinterpret_cast<float4*>(static_cast<uint8_t*>(a.out) + b * bytes);
 #pragma unroll 4
-  for (int i = lane; i < kQHeads * kDim / 4; i += 32) d[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = lane; i < bytes / 16; i += 32) d[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Output rows of (sequence b, kv head g).
+__device__ __forceinline__ OutRows out_rows(const DecodeArgs& a, int b, int g) {
+  const int64_t e = (static_cast<int64_t>(b) * a.num_queries * kQHeads + g * kGroup) * kDim;
+  void* base = a.out_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.out) + e)
+                          : static_cast<void*>(static_cast<float*>(a.out) + e);
+  return OutRows{base, kQHeads * kDim, a.out_bf16 != 0};
 }
 
 // Fixed-order log-sum-exp merge of `cnt` partial records P[0], P[stride],
 // ... (pieces of one (sequence, kv head) unit, in piece order):
 //   M[h] = max_s m_s[h],  w_s[h] = exp2(m_s[h] - M[h]),
 //   S[h] = sum_s w_s[h] l_s[h],  O[h][d] = sum_s w_s[h] acc_s[h][d].
-// With `final`, out[h][d] = O / S (zero where S == 0); otherwise (M, S, O)
-// is written as one partial record at `out`.  Pieces are taken 32 at a time
+// With `final_out`, query final_q's rows of it get O / S (zero where S == 0);
+// otherwise (M, S, O) is written as one partial record at `out`.  Pieces are taken 32 at a time
 // (running max rescaled between groups, a fixed order): lane s reads m and l
 // of piece s, and every lane accumulates dims 2*lane, 2*lane+1 of the 4 heads
 // with the loads of kMergeBatch pieces in flight.  kShared: P lives in shared
@@ -547,7 +631,8 @@ __device__ __forceinline__ float2 ld2(const float* p) {
 
 template <bool kShared>
 __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stride, float* out,
-                                               bool final, int lane) {
+                                               const OutRows* final_out, int final_q, int lane) {
+  const bool final = final_out != nullptr;
   const int64_t step = static_cast<int64_t>(stride) * kPartialFloats;
   float M[kGroup], S[kGroup];
   float2 O[kGroup];
@@ -621,7 +706,7 @@ __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stri
 #pragma unroll
     for (int h = 0; h < kGroup; ++h) {
       const float inv = S[h] > 0.f ? 1.f / S[h] : 0.f;
-      reinterpret_cast<float2*>(out + h * kDim)[lane] = make_float2(O[h].x * inv, O[h].y * inv);
+      final_out->put2(final_q, h, 2 * lane, O[h].x * inv, O[h].y * inv);
     }
   } else {
     if (lane == 0) {
@@ -665,11 +750,11 @@ __device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a,
                                            const int32_t* s_pfx, int b, int g, int j0, int j1,
                                            int np, int64_t chunk, int lane) {
   if (j0 == 0 && j1 == np - 1) {
-    cmp.finalize(a.out + (static_cast<int64_t>(b) * kQHeads + g * kGroup) * kDim, lane);
+    cmp.finalize(out_rows(a, b, g), a.num_queries, lane);
     return;
   }
   const int64_t slot = static_cast<int64_t>(g) * (a.batch + gridDim.x) + b + blockIdx.x;
-  cmp.store_partial(a.partials + slot * kPartialFloats, lane);
+  cmp.store_partial(a.partials + slot * a.num_queries * kPartialFloats, a.num_queries, lane);
 }
 
 // Producer-side description of page f (this lane's slot of a 32-page batch):
@@ -693,6 +778,7 @@ template <class C>
 struct SmemPlan {
   static constexpr int S = C::kStages;
   static constexpr size_t stages = 0;   // [S][page 32 KiB | query rows 4 KiB]
+  static constexpr int kStageBytes = StageLayout<C::kQueries>::kBytes;
   static constexpr size_t scratch = stages + size_t(S) * kStageBytes;
   static constexpr size_t full = scratch + size_t(kWarps) * kScratchBytes;
   static constexpr size_t empty = full + size_t(S) * 8;
@@ -719,6 +805,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   volatile int32_t* s_flags = reinterpret_cast<int32_t*>(smem + L::flags);
   volatile int32_t* s_phys = reinterpret_cast<int32_t*>(smem + L::phys);
   const bool fused = a.k_new != nullptr;
+  constexpr int nq = C::kQueries;   // == a.num_queries (the host picks the variant)
   int32_t* s_len = reinterpret_cast<int32_t*>(smem + L::lens);
   int32_t* s_pfx = s_len + B;
   const uint32_t base = smem_addr(smem);
@@ -765,7 +852,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
 
   // empty (or invalid) sequences: zero output rows, once across the grid
   for (int b = blockIdx.x * kWarps + warp; b < B; b += G * kWarps)
-    if (s_pfx[b + 1] == s_pfx[b]) zero_rows(a.out + static_cast<int64_t>(b) * kQHeads * kDim, lane);
+    if (s_pfx[b + 1] == s_pfx[b]) zero_rows(a, b, lane);
   if (n <= 0) return;
   // Issue page r into stage r % kS (warp 0 only; stage known to be free).
   // Test-only: leave page 0's full barrier unarmed, so the consumers' bounded
@@ -785,7 +872,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
     if (lane == 0 && !(stall && r == 0)) {
       const int st = r % kS;
       const uint32_t bar = full + 8 * st;
-      const uint32_t dst = base + L::stages + st * kStageBytes;
+      const uint32_t dst = base + L::stages + st * L::kStageBytes;
       const bool ok = static_cast<uint32_t>(phys) < static_cast<uint32_t>(a.num_pages);
       const bool start = info & 1;
       const bool append = fused && (info & 2);
@@ -794,13 +881,14 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
       s_phys[st] = phys;
       if (!ok) record_error(a.err, kErrBadPage);
       const uint32_t bytes =
-          (ok ? kPageBytes : 0) + (start ? kQRowsBytes : 0) + (append ? kNewRowsBytes : 0);
+          (ok ? kPageBytes : 0) + (start ? nq * kQRowsBytes : 0) + (append ? kNewRowsBytes : 0);
       if (bytes) {
         mbar_arrive_expect_tx(bar, bytes);
         if (ok) tma_load_tile(dst, &tmap, 0, phys * kRowsPerPage, bar, policy);
-        if (start) bulk_load(dst + kPageBytes, a.q + seq * kQHeads * kDim, kQRowsBytes, bar);
+        if (start)
+          bulk_load(dst + kPageBytes, a.q + seq * nq * kQHeads * kDim, nq * kQRowsBytes, bar);
         if (append) {
-          const uint32_t nd = dst + kPageBytes + kQRowsBytes;
+          const uint32_t nd = dst + kPageBytes + nq * kQRowsBytes;
           bulk_load(nd, a.k_new + seq * kKvHeads * kDim, kNewRowsBytes / 2, bar);
           bulk_load(nd + kNewRowsBytes / 2, a.v_new + seq * kKvHeads * kDim, kNewRowsBytes / 2,
                     bar);
@@ -857,9 +945,9 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
       drain(r + 1);
       return;
     }
-    const uint32_t stage = base + L::stages + st * kStageBytes;
+    const uint32_t stage = base + L::stages + st * L::kStageBytes;
     if (need_q) {
-      cmp.begin(stage + kPageBytes + warp * (kGroup * kRowBytes), lane);
+      cmp.begin(stage + kPageBytes, warp, nq, lane);
       need_q = false;
     }
     if (fused && j == np - 1) {
@@ -868,7 +956,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
       if (lane < 16) {
         const int kv = lane >> 3, c = lane & 7;
         const int slot = (Lb - 1) % kTokens;
-        const uint4 v = lds128(stage + kPageBytes + kQRowsBytes + kv * (kNewRowsBytes / 2) +
+        const uint4 v = lds128(stage + kPageBytes + nq * kQRowsBytes + kv * (kNewRowsBytes / 2) +
                                warp * kRowBytes + c * 16);
         const int row = kv * (kKvHeads * kTokens) + warp * kTokens + slot;
         sts128(stage + swz(row, c), v);
@@ -882,9 +970,13 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
       __syncwarp();
     }
     if (!s_flags[st]) {
+      // tokens of this page in the context of the last query, and of the
+      // first of two (whose context ends one token earlier)
       const int nvalid = min(kTokens, Lb - kTokens * j);
+      const int nvalid_q0 = nq == 1 ? nvalid : min(kTokens, Lb - 1 - kTokens * j);
       const uint32_t ktile = stage + warp * kTileBytes;
-      cmp.consume(ktile, ktile + kKvHeads * kTileBytes, scratch, nvalid, a.scale_log2, lane);
+      cmp.consume(ktile, ktile + kKvHeads * kTileBytes, scratch, nvalid, nvalid_q0, a.scale_log2,
+                  lane);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + 8 * st);
@@ -928,7 +1020,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   int before = 0, all = 0;
   for (int i = threadIdx.x; i < a.batch; i += blockDim.x) {
     int L = a.seq_lens[i];
-    if (L < 0 || L > cap) L = 0;
+    if (L < 0 || L > cap || (L > 0 && L < a.num_queries)) L = 0;
     const int np = (L + kTokens - 1) / kTokens;
     all += np;
     before += (i < b) ? np : 0;
@@ -950,24 +1042,31 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
     pages_all += s_sum[1][k];
   }
   int Lb = a.seq_lens[b];
-  if (Lb < 0 || Lb > cap) Lb = 0;
+  if (Lb < 0 || Lb > cap || (Lb > 0 && Lb < a.num_queries)) Lb = 0;
   const int64_t chunk = range_chunk(pages_all, a.batch, decode_grid, a.min_chunk);
   const int2 sp = split_of(pages_before, b, (Lb + kTokens - 1) / kTokens, chunk);
   const int K = sp.y;
-  if (K <= 1) return;
+  // This grid's completion is what the next programmatically dependent
+  // launch waits for, so it must imply decode's: CTA (0, 0) always waits for
+  // the decode grid; the other CTAs without work leave at once, freeing
+  // their SM slot for the next launch.
+  if (K <= 1 && (g | b) != 0) return;
   pdl_wait();   // the pieces are written by the decode grid
+  if (K <= 1) return;
+  const int nq = a.num_queries;
   const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + sp.x;
   const int parts = min(kMergeWarps, K);
-  if (warp < parts) {
-    const int cnt = (K - warp + kMergeWarps - 1) / kMergeWarps;
-    merge_partials<false>(a.partials + (S0 + warp) * kPartialFloats, cnt, kMergeWarps,
-                          s_part[warp], false, lane);
+  const OutRows out = out_rows(a, b, g);
+  for (int qi = 0; qi < nq; ++qi) {   // a piece's record of query qi: slot * nq + qi
+    if (warp < parts) {
+      const int cnt = (K - warp + kMergeWarps - 1) / kMergeWarps;
+      merge_partials<false>(a.partials + ((S0 + warp) * nq + qi) * kPartialFloats, cnt,
+                            kMergeWarps * nq, s_part[warp], nullptr, 0, lane);
+    }
+    __syncthreads();
+    if (warp == 0) merge_partials<true>(&s_part[0][0], parts, 1, nullptr, &out, qi, lane);
+    __syncthreads();   // s_part is rewritten for the next query
   }
-  __syncthreads();
-  if (warp == 0)
-    merge_partials<true>(&s_part[0][0], parts, 1,
-                         a.out + (static_cast<int64_t>(b) * kQHeads + g * kGroup) * kDim, true,
-                         lane);
 }
 
 // ---------------------------------------------------------------- host side --
@@ -977,28 +1076,31 @@ static const void* kernel_ptr() {
   return reinterpret_cast<const void*>(&decode_kernel<C>);
 }
 
-static const void* kernel_for(int kernel) {
-  switch (kernel) {
-    case PKV_KERNEL_SIMT: return kernel_ptr<SimtCompute>();
-    case PKV_KERNEL_MMA: return kernel_ptr<MmaCompute>();
-    default: return nullptr;
-  }
+using MmaCompute1 = MmaComputeT<1>;
+using MmaCompute2 = MmaComputeT<2>;
+
+static const void* kernel_for(int kernel, int nq) {
+  if (kernel == PKV_KERNEL_SIMT) return nq == 1 ? kernel_ptr<SimtCompute>() : nullptr;
+  if (kernel == PKV_KERNEL_MMA)
+    return nq == 1 ? kernel_ptr<MmaCompute1>() : nq == 2 ? kernel_ptr<MmaCompute2>() : nullptr;
+  return nullptr;
 }
 
-static size_t smem_for(int kernel, int32_t batch) {
-  return kernel == PKV_KERNEL_SIMT ? SmemPlan<SimtCompute>::bytes(batch)
-                                   : SmemPlan<MmaCompute>::bytes(batch);
+static size_t smem_for(int kernel, int nq, int32_t batch) {
+  if (kernel == PKV_KERNEL_SIMT) return SmemPlan<SimtCompute>::bytes(batch);
+  return nq == 2 ? SmemPlan<MmaCompute2>::bytes(batch) : SmemPlan<MmaCompute1>::bytes(batch);
 }
 
 cudaError_t prepare_decode_kernels(int device) {
   int optin = 0;
   cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
   if (e != cudaSuccess) return e;
-  for (int k : {PKV_KERNEL_SIMT, PKV_KERNEL_MMA}) {
+  for (const void* fn : {kernel_for(PKV_KERNEL_SIMT, 1), kernel_for(PKV_KERNEL_MMA, 1),
+                          kernel_for(PKV_KERNEL_MMA, 2)}) {
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, kernel_for(k));
+    e = cudaFuncGetAttributes(&fa, fn);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kernel_for(k), cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              optin - static_cast<int>(fa.sharedSizeBytes));
     if (e != cudaSuccess) return e;
   }
@@ -1006,15 +1108,16 @@ cudaError_t prepare_decode_kernels(int device) {
 }
 
 int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,
-                DecodePlan* plan) {
+                int num_queries, DecodePlan* plan) {
+  if (num_queries < 1 || num_queries > kMaxQueries) return PKV_ERR_UNSUPPORTED;
   if (kernel == PKV_KERNEL_AUTO) kernel = PKV_KERNEL_MMA;
-  const void* fn = kernel_for(kernel);
+  const void* fn = kernel_for(kernel, num_queries);
   if (!fn) return PKV_ERR_UNSUPPORTED;
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) !=
       cudaSuccess)
     return PKV_ERR_CUDA;
-  const size_t smem = smem_for(kernel, batch);
+  const size_t smem = smem_for(kernel, num_queries, batch);
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return PKV_ERR_CUDA;
   if (smem + fa.sharedSizeBytes > static_cast<size_t>(optin)) return PKV_ERR_UNSUPPORTED;
@@ -1023,11 +1126,12 @@ int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ct
     return PKV_ERR_CUDA;
   if (per_sm < 1) return PKV_ERR_UNSUPPORTED;
   plan->kernel = kernel;
+  plan->num_queries = num_queries;
   plan->threads = kWarps * 32;
   plan->smem = smem;
   plan->grid = grid_ctas > 0 ? grid_ctas : sm_count * per_sm;
   const int64_t slots = static_cast<int64_t>(kKvHeads) * (batch + plan->grid);
-  plan->ws_bytes = static_cast<size_t>(slots) * kPartialFloats * sizeof(float);
+  plan->ws_bytes = static_cast<size_t>(slots) * num_queries * kPartialFloats * sizeof(float);
   return PKV_OK;
 }
 
@@ -1052,7 +1156,10 @@ cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const
   cudaError_t e;
   switch (plan.kernel) {
     case PKV_KERNEL_SIMT: e = launch_one<SimtCompute>(plan, tmap, a, flags, stream); break;
-    case PKV_KERNEL_MMA: e = launch_one<MmaCompute>(plan, tmap, a, flags, stream); break;
+    case PKV_KERNEL_MMA:
+      e = plan.num_queries == 2 ? launch_one<MmaCompute2>(plan, tmap, a, flags, stream)
+                                : launch_one<MmaCompute1>(plan, tmap, a, flags, stream);
+      break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;

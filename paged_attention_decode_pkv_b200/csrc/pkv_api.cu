@@ -215,7 +215,7 @@ int pkv_decode_workspace_bytes_ex(const pkv_pool* pool, int32_t batch, int32_t k
                                   int32_t grid_ctas, size_t* bytes_out) {
   if (!pool || !bytes_out || batch < 0 || grid_ctas < 0) return PKV_ERR_INVALID_ARG;
   pkv::DecodePlan plan;
-  int s = pkv::plan_decode(pool->device, pool->sm_count, batch, kernel, grid_ctas, &plan);
+  int s = pkv::plan_decode(pool->device, pool->sm_count, batch, kernel, grid_ctas, 1, &plan);
   if (s != PKV_OK) return s;
   *bytes_out = plan.ws_bytes;
   return PKV_OK;
@@ -232,17 +232,22 @@ namespace {
 // Decode, with the fused append when k_new / v_new are given.
 int decode_common(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
                   const pkv_pool* pool, const int32_t* block_tables, const int32_t* seq_lens,
-                  int32_t layer, float scale, float* out, int32_t num_layers, int32_t batch,
-                  int32_t max_blocks, void* workspace, size_t workspace_bytes,
-                  pkv_stream_t stream, int32_t kernel, int32_t grid_ctas, int32_t min_chunk) {
+                  int32_t layer, float scale, void* out, int32_t out_dtype, int32_t num_queries,
+                  int32_t num_layers, int32_t batch, int32_t max_blocks, void* workspace,
+                  size_t workspace_bytes, pkv_stream_t stream, int32_t kernel, int32_t grid_ctas,
+                  int32_t min_chunk) {
   int s = check_table_args(pool, block_tables, seq_lens, layer, num_layers, batch, max_blocks);
   if (s != PKV_OK) return s;
   if (!q || !out || !aligned(q, 16) || !aligned(out, 16)) return PKV_ERR_INVALID_ARG;
   if (!(scale == scale) || grid_ctas < 0 || min_chunk < 0) return PKV_ERR_INVALID_ARG;
-  if (batch == 0) return PKV_OK;
+  if (out_dtype != PKV_DTYPE_F32 && out_dtype != PKV_DTYPE_BF16) return PKV_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return PKV_ERR_INVALID_ARG;
+  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16))) return PKV_ERR_INVALID_ARG;
+  if (k_new && num_queries != 1) return PKV_ERR_UNSUPPORTED;
   pkv::DecodePlan plan;
-  s = pkv::plan_decode(pool->device, pool->sm_count, batch, kernel, grid_ctas, &plan);
+  s = pkv::plan_decode(pool->device, pool->sm_count, batch, kernel, grid_ctas, num_queries, &plan);
   if (s != PKV_OK) return s;
+  if (batch == 0) return PKV_OK;
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < plan.ws_bytes)
     return PKV_ERR_WORKSPACE;
   pkv::DecodeArgs a;
@@ -258,6 +263,8 @@ int decode_common(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_ne
   a.min_chunk = min_chunk;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.flags = pool->launch_flags;
+  a.num_queries = num_queries;
+  a.out_bf16 = out_dtype == PKV_DTYPE_BF16;
   a.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
   a.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
   a.pool = static_cast<__nv_bfloat16*>(pool->data);
@@ -276,8 +283,8 @@ int paged_attention_decode_ex(const uint16_t* q, const pkv_pool* pool,
                               pkv_stream_t stream, int32_t kernel, int32_t grid_ctas,
                               int32_t min_chunk) {
   return decode_common(q, nullptr, nullptr, pool, block_tables, seq_lens, layer, scale, out,
-                       num_layers, batch, max_blocks, workspace, workspace_bytes, stream, kernel,
-                       grid_ctas, min_chunk);
+                       PKV_DTYPE_F32, 1, num_layers, batch, max_blocks, workspace, workspace_bytes,
+                       stream, kernel, grid_ctas, min_chunk);
 }
 
 int paged_attention_decode_append_ex(const uint16_t* q, const uint16_t* k_new,
@@ -287,10 +294,31 @@ int paged_attention_decode_append_ex(const uint16_t* q, const uint16_t* k_new,
                                      int32_t batch, int32_t max_blocks, void* workspace,
                                      size_t workspace_bytes, pkv_stream_t stream, int32_t kernel,
                                      int32_t grid_ctas, int32_t min_chunk) {
-  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return PKV_ERR_INVALID_ARG;
+  if (!k_new || !v_new) return PKV_ERR_INVALID_ARG;
   return decode_common(q, k_new, v_new, pool, block_tables, seq_lens, layer, scale, out,
-                       num_layers, batch, max_blocks, workspace, workspace_bytes, stream, kernel,
-                       grid_ctas, min_chunk);
+                       PKV_DTYPE_F32, 1, num_layers, batch, max_blocks, workspace, workspace_bytes,
+                       stream, kernel, grid_ctas, min_chunk);
+}
+
+int pkv_decode(pkv_pool* pool, const pkv_decode_params* p, pkv_stream_t stream) {
+  if (!p || p->struct_size < sizeof(pkv_decode_params)) return PKV_ERR_INVALID_ARG;
+  return decode_common(p->q, p->k_new, p->v_new, pool, p->block_tables, p->seq_lens, p->layer,
+                       p->scale, p->out, p->out_dtype, p->num_queries, p->num_layers, p->batch,
+                       p->max_blocks, p->workspace, p->workspace_bytes, stream, p->kernel,
+                       p->grid_ctas, p->min_chunk);
+}
+
+int pkv_decode_params_workspace_bytes(const pkv_pool* pool, const pkv_decode_params* p,
+                                      size_t* bytes_out) {
+  if (!pool || !p || !bytes_out || p->struct_size < sizeof(pkv_decode_params) || p->batch < 0 ||
+      p->grid_ctas < 0)
+    return PKV_ERR_INVALID_ARG;
+  pkv::DecodePlan plan;
+  int s = pkv::plan_decode(pool->device, pool->sm_count, p->batch, p->kernel, p->grid_ctas,
+                           p->num_queries, &plan);
+  if (s != PKV_OK) return s;
+  *bytes_out = plan.ws_bytes;
+  return PKV_OK;
 }
 
 int paged_attention_decode_append(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,

@@ -24,6 +24,7 @@ constexpr int kRowBytes = kDim * 2;               // one token of one kv head: 1
 constexpr int kTileBytes = kTokens * kRowBytes;   // (page, K|V, kv head) tile: 2 KiB
 constexpr int kRowsPerPage = 2 * kKvHeads * kTokens;  // 256 rows of 128 B
 constexpr int kPartialFloats = 2 * kGroup + kGroup * kDim;  // m[4], l[4], acc[4][64]
+constexpr int kMaxQueries = 2;   // queries per sequence in one decode launch
 
 // Sticky device error codes (first one wins).
 constexpr int32_t kErrBadPage = PKV_ERR_BAD_PAGE;
@@ -207,8 +208,8 @@ struct DecodeArgs {
   const __nv_bfloat16* q;   // [B][32][64]
   const int32_t* bt;        // this layer's block-table slab [B][max_blocks]
   const int32_t* seq_lens;  // [B]
-  float* out;               // [B][32][64]
-  float* partials;          // [8 kv heads][B + grid][kPartialFloats]
+  void* out;                // [B][num_queries][32][64], FP32 or BF16 (out_bf16)
+  float* partials;          // [8 kv heads][B + grid][num_queries][kPartialFloats]
   int32_t* err;             // sticky device error word
   int32_t batch;
   int32_t max_blocks;
@@ -216,6 +217,8 @@ struct DecodeArgs {
   int32_t min_chunk;        // minimum pages per CTA range
   float scale_log2;         // scale * log2(e)
   int32_t flags;            // kLaunch* bits
+  int32_t num_queries;      // queries per sequence (1 or kMaxQueries), causal among them
+  int32_t out_bf16;         // nonzero: out is BF16
   // Fused append (paged_attention_decode_append): the new token's K/V rows
   // [B][8][64] and the page storage they are written into; null otherwise.
   const __nv_bfloat16* k_new;
@@ -226,6 +229,7 @@ struct DecodeArgs {
 // Launch planning shared by the workspace query and the launch.
 struct DecodePlan {
   int kernel;        // PKV_KERNEL_SIMT or PKV_KERNEL_MMA
+  int num_queries;   // queries per sequence (picks the kernel variant)
   int grid;          // CTAs
   int threads;       // threads per CTA
   size_t smem;       // dynamic shared memory bytes
@@ -233,7 +237,7 @@ struct DecodePlan {
 };
 
 int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,
-                DecodePlan* plan);
+                int num_queries, DecodePlan* plan);
 cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const DecodeArgs& a,
                           int flags, cudaStream_t stream);
 cudaError_t prepare_decode_kernels(int device);

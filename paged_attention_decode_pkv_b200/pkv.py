@@ -24,6 +24,8 @@ HEAD_DIM = 64
 PAGE_BYTES = 32768
 
 KERNEL_AUTO, KERNEL_SIMT, KERNEL_MMA = 0, 1, 2
+DTYPE_F32, DTYPE_BF16 = 0, 1
+MAX_QUERIES = 2
 LAUNCH_PDL = 1
 LAUNCH_EARLY_TABLES = 2
 LAUNCH_TEST_STALL = 1 << 30
@@ -47,8 +49,22 @@ EXPORTS = (
     "pkv_last_error_message", "pkv_pool_set_launch_flags", "paged_attention_decode_noalloc",
     "pkv_fill", "pkv_allocator_create", "pkv_allocator_destroy", "pkv_allocator_free_count",
     "pkv_allocator_alloc", "pkv_allocator_free", "paged_attention_decode_append",
-    "paged_attention_decode_append_ex",
+    "paged_attention_decode_append_ex", "pkv_decode", "pkv_decode_params_workspace_bytes",
 )
+
+
+class DecodeParams(ctypes.Structure):
+    """pkv_decode_params (include/pkv.h), field for field."""
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t), ("q", ctypes.c_void_p), ("k_new", ctypes.c_void_p),
+        ("v_new", ctypes.c_void_p), ("block_tables", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p), ("out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t), ("scale", ctypes.c_float),
+        ("layer", ctypes.c_int32), ("num_layers", ctypes.c_int32), ("batch", ctypes.c_int32),
+        ("max_blocks", ctypes.c_int32), ("num_queries", ctypes.c_int32),
+        ("out_dtype", ctypes.c_int32), ("kernel", ctypes.c_int32), ("grid_ctas", ctypes.c_int32),
+        ("min_chunk", ctypes.c_int32),
+    ]
 
 
 def _load():
@@ -81,6 +97,9 @@ def _load():
                                            i32, P, sz, P], ctypes.c_int),
         "paged_attention_decode_append_ex": ([P, P, P, P, P, P, i32, ctypes.c_float, P, i32, i32,
                                               i32, P, sz, P, i32, i32, i32], ctypes.c_int),
+        "pkv_decode": ([P, ctypes.POINTER(DecodeParams), P], ctypes.c_int),
+        "pkv_decode_params_workspace_bytes": ([P, ctypes.POINTER(DecodeParams),
+                                               ctypes.POINTER(sz)], ctypes.c_int),
         "pkv_allocator_create": ([i32, ctypes.POINTER(P)], ctypes.c_int),
         "pkv_allocator_destroy": ([P], ctypes.c_int),
         "pkv_allocator_free_count": ([P], i32),
@@ -194,13 +213,27 @@ class Pool:
                    "pkv_decode_workspace_bytes")
         return n.value
 
-    def workspace(self, batch: int, kernel: int = KERNEL_AUTO, grid_ctas: int = 0) -> torch.Tensor:
-        """A decode workspace, cached per (batch, kernel, grid)."""
-        key = (int(batch), int(kernel), int(grid_ctas))
+    def workspace_bytes_for(self, batch: int, num_queries: int = 1, kernel: int = KERNEL_AUTO,
+                            grid_ctas: int = 0) -> int:
+        p = DecodeParams(struct_size=ctypes.sizeof(DecodeParams), batch=int(batch),
+                         num_queries=int(num_queries), kernel=int(kernel),
+                         grid_ctas=int(grid_ctas))
+        n = ctypes.c_size_t()
+        with torch.cuda.device(self.device):
+            _check(lib.pkv_decode_params_workspace_bytes(self.handle, ctypes.byref(p),
+                                                         ctypes.byref(n)),
+                   "pkv_decode_params_workspace_bytes")
+        return n.value
+
+    def workspace(self, batch: int, kernel: int = KERNEL_AUTO, grid_ctas: int = 0,
+                  num_queries: int = 1) -> torch.Tensor:
+        """A decode workspace, cached per (batch, kernel, grid, queries)."""
+        key = (int(batch), int(kernel), int(grid_ctas), int(num_queries))
         ws = self._ws.get(key)
         if ws is None:
-            ws = torch.zeros(max(256, self.workspace_bytes(*key)), dtype=torch.uint8,
-                             device=self.device)
+            n = (self.workspace_bytes(*key[:3]) if num_queries == 1 else
+                 self.workspace_bytes_for(batch, num_queries, kernel, grid_ctas))
+            ws = torch.zeros(max(256, n), dtype=torch.uint8, device=self.device)
             self._ws[key] = ws
         return ws
 
@@ -255,6 +288,42 @@ def decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, poo
         _dev(out, torch.float32, (B, NUM_Q_HEADS, HEAD_DIM), "out"), L, B, MB,
         _dev(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream),
         int(kernel), int(grid_ctas), int(min_chunk)), "paged_attention_decode_append")
+    return out
+
+
+def decode_general(q: torch.Tensor, pool: Pool, block_tables: torch.Tensor,
+                   seq_lens: torch.Tensor, layer: int, scale: float, num_queries: int = 1,
+                   out_dtype=torch.float32, out: Optional[torch.Tensor] = None,
+                   k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, kernel: int = KERNEL_AUTO,
+                   grid_ctas: int = 0, min_chunk: int = 0, stream=None) -> torch.Tensor:
+    """pkv_decode: q and out are [B, num_queries, 32, 64] ([B, 32, 64] when
+    num_queries is 1); out_dtype torch.float32 or torch.bfloat16."""
+    L, B, MB = block_tables.shape
+    T = int(num_queries)
+    shape = (B, NUM_Q_HEADS, HEAD_DIM) if T == 1 else (B, T, NUM_Q_HEADS, HEAD_DIM)
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out_dtype must be torch.float32 or torch.bfloat16")
+    if out is None:
+        out = torch.empty(shape, dtype=out_dtype, device=q.device)
+    if workspace is None:
+        workspace = pool.workspace(B, kernel, grid_ctas, T)
+    p = DecodeParams(struct_size=ctypes.sizeof(DecodeParams))
+    p.q = _dev(q, torch.bfloat16, shape, "q")
+    if k_new is not None or v_new is not None:
+        p.k_new = _dev(k_new, torch.bfloat16, (B, NUM_KV_HEADS, HEAD_DIM), "k_new")
+        p.v_new = _dev(v_new, torch.bfloat16, (B, NUM_KV_HEADS, HEAD_DIM), "v_new")
+    p.block_tables = _dev(block_tables, torch.int32, None, "block_tables")
+    p.seq_lens = _dev(seq_lens, torch.int32, (B,), "seq_lens")
+    p.out = _dev(out, out_dtype, shape, "out")
+    p.workspace = _dev(workspace, torch.uint8, None, "workspace")
+    p.workspace_bytes = workspace.numel()
+    p.scale = float(scale)
+    p.layer, p.num_layers, p.batch, p.max_blocks = int(layer), L, B, MB
+    p.num_queries = T
+    p.out_dtype = DTYPE_BF16 if out_dtype == torch.bfloat16 else DTYPE_F32
+    p.kernel, p.grid_ctas, p.min_chunk = int(kernel), int(grid_ctas), int(min_chunk)
+    _check(lib.pkv_decode(pool.handle, ctypes.byref(p), _stream(stream)), "pkv_decode")
     return out
 
 

@@ -66,3 +66,22 @@ def test_calls_reject_null_pool():
     assert pkv.lib.pkv_pool_destroy(None) == pkv.OK
     assert pkv.lib.pkv_pool_num_pages(None) == -1
     assert pkv.lib.pkv_fill(None, P, P, P, P, P, 16, 0, 1, 1, 1, None) == pkv.ERR_INVALID_ARG
+
+
+def test_decode_params_struct_matches_the_header(tmp_path):
+    # the binding's ctypes mirror of pkv_decode_params must have the C layout
+    from paged_attention_decode_pkv_b200 import pkv
+    import subprocess
+    fields = [f[0] for f in pkv.DecodeParams._fields_]
+    src = ["#include <stdio.h>", "#include <stddef.h>", '#include "pkv.h"', "int main(void) {",
+           '  printf("%zu\\n", sizeof(pkv_decode_params));']
+    src += ['  printf("%%zu\\n", offsetof(pkv_decode_params, %s));' % f for f in fields]
+    src += ["  return 0;", "}"]
+    (tmp_path / "layout.c").write_text("\n".join(src))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(tmp_path / "layout.c"),
+                    "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(pkv.DecodeParams)
+    assert got[1:] == [getattr(pkv.DecodeParams, f).offset for f in fields]
