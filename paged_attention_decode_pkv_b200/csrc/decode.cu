@@ -52,6 +52,8 @@
 //    costs no accuracy; softmax stays FP32 on the CUDA cores.  The MMA's
 //    N = 8 holds 4 heads; with n = 2 the other 4 columns carry a second query
 //    of the same sequence (causal: it sees one token more than the first).
+#include <type_traits>
+
 #include "pkv_internal.cuh"
 
 namespace pkv {
@@ -79,25 +81,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // Output rows of one (sequence, kv head) unit: element (query i, head h of
-// the group, dim d) is at base + i * qstride + h * 64 + d, FP32 or BF16
-// (rounded to nearest even).  Partial records use the same shape in FP32.
-struct OutRows {
+// the group, dim d) is at base + i * qstride + h * 64 + d, FP32 or (kBf16)
+// BF16 rounded to nearest even.  Partial records use the same shape in FP32.
+template <bool kBf16>
+struct OutRowsT {
   void* base;
   int64_t qstride;   // elements
-  bool bf16;
 
   __device__ __forceinline__ int64_t at(int i, int h, int d) const {
     return i * qstride + h * kDim + d;
   }
   __device__ __forceinline__ void put(int i, int h, int d, float v) const {
-    if (bf16)
+    if constexpr (kBf16)
       static_cast<__nv_bfloat16*>(base)[at(i, h, d)] = __float2bfloat16_rn(v);
     else
       static_cast<float*>(base)[at(i, h, d)] = v;
   }
   // dims d, d + 1 (d even)
   __device__ __forceinline__ void put2(int i, int h, int d, float x, float y) const {
-    if (bf16)
+    if constexpr (kBf16)
       *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(base) + at(i, h, d)) =
           pack_bf16x2(x, y);
     else
@@ -105,7 +107,7 @@ struct OutRows {
   }
   // dims d .. d + 7 (d a multiple of 8)
   __device__ __forceinline__ void put8(int i, int h, int d, const float* v) const {
-    if (bf16) {
+    if constexpr (kBf16) {
       *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + at(i, h, d)) =
           make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
                      pack_bf16x2(v[6], v[7]));
@@ -305,7 +307,8 @@ struct SimtCompute {
     l[3] = b2 ? s2[1] : o1;
   }
 
-  __device__ __forceinline__ void finalize(const OutRows& out, int /*nq*/, int lane) const {
+  template <class Out>
+  __device__ __forceinline__ void finalize(const Out& out, int lane) const {
     float r[8], l[4];
     const int h = reduce_acc(r, lane);
     reduce_l(l, lane);
@@ -481,7 +484,8 @@ struct MmaComputeT {
 
   // O^T columns 2qd, 2qd + 1 = query qd / 2, heads 2(qd % 2), 2(qd % 2) + 1,
   // scaled by s0, s1; lanes whose query does not exist write nothing.
-  __device__ __forceinline__ void write_rows(const OutRows& out, int /*nq*/, int lane, float s0,
+  template <class Out>
+  __device__ __forceinline__ void write_rows(const Out& out, int lane, float s0,
                                              float s1) const {
     constexpr int nq = kNq;
     const int r = lane >> 2, qd = lane & 3;
@@ -497,10 +501,11 @@ struct MmaComputeT {
     }
   }
 
-  __device__ __forceinline__ void finalize(const OutRows& out, int nq, int lane) const {
+  template <class Out>
+  __device__ __forceinline__ void finalize(const Out& out, int lane) const {
     float l0, l1;
     reduce_l(l0, l1);
-    write_rows(out, nq, lane, 1.f / l0, 1.f / l1);
+    write_rows(out, lane, 1.f / l0, 1.f / l1);
   }
 
   // Partial records, one per query: P + i * kPartialFloats = m[4], l[4],
@@ -517,7 +522,7 @@ struct MmaComputeT {
       rec[kGroup + h] = l0;
       rec[kGroup + h + 1] = l1;
     }
-    write_rows(OutRows{P + 2 * kGroup, kPartialFloats, false}, nq, lane, 1.f, 1.f);
+    write_rows(OutRowsT<false>{P + 2 * kGroup, kPartialFloats}, lane, 1.f, 1.f);
   }
 };
 
@@ -601,11 +606,11 @@ __device__ __forceinline__ void zero_rows(const DecodeArgs& a, int b, int lane) 
 }
 
 // Output rows of (sequence b, kv head g).
-__device__ __forceinline__ OutRows out_rows(const DecodeArgs& a, int b, int g) {
+template <bool kBf16>
+__device__ __forceinline__ OutRowsT<kBf16> out_rows(const DecodeArgs& a, int b, int g) {
   const int64_t e = (static_cast<int64_t>(b) * a.num_queries * kQHeads + g * kGroup) * kDim;
-  void* base = a.out_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.out) + e)
-                          : static_cast<void*>(static_cast<float*>(a.out) + e);
-  return OutRows{base, kQHeads * kDim, a.out_bf16 != 0};
+  using T = typename std::conditional<kBf16, __nv_bfloat16, float>::type;
+  return OutRowsT<kBf16>{static_cast<T*>(a.out) + e, kQHeads * kDim};
 }
 
 // Fixed-order log-sum-exp merge of `cnt` partial records P[0], P[stride],
@@ -629,9 +634,9 @@ __device__ __forceinline__ float2 ld2(const float* p) {
   return kShared ? *reinterpret_cast<const float2*>(p) : __ldcg(reinterpret_cast<const float2*>(p));
 }
 
-template <bool kShared>
+template <bool kShared, class Out>
 __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stride, float* out,
-                                               const OutRows* final_out, int final_q, int lane) {
+                                               const Out* final_out, int final_q, int lane) {
   const bool final = final_out != nullptr;
   const int64_t step = static_cast<int64_t>(stride) * kPartialFloats;
   float M[kGroup], S[kGroup];
@@ -750,7 +755,10 @@ __device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a,
                                            const int32_t* s_pfx, int b, int g, int j0, int j1,
                                            int np, int64_t chunk, int lane) {
   if (j0 == 0 && j1 == np - 1) {
-    cmp.finalize(out_rows(a, b, g), a.num_queries, lane);
+    if (a.out_bf16)
+      cmp.finalize(out_rows<true>(a, b, g), lane);
+    else
+      cmp.finalize(out_rows<false>(a, b, g), lane);
     return;
   }
   const int64_t slot = static_cast<int64_t>(g) * (a.batch + gridDim.x) + b + blockIdx.x;
@@ -1009,6 +1017,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
 // ---------------------------------------------------------------------------
 constexpr int kMergeWarps = 8;
 
+template <int kNq, bool kBf16>
 __global__ void __launch_bounds__(kMergeWarps * 32)
     merge_kernel(const DecodeArgs a, int32_t decode_grid) {
   __shared__ __align__(16) float s_part[kMergeWarps][kPartialFloats];
@@ -1053,19 +1062,21 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   if (K <= 1 && (g | b) != 0) return;
   pdl_wait();   // the pieces are written by the decode grid
   if (K <= 1) return;
-  const int nq = a.num_queries;
+  constexpr int nq = kNq;   // == a.num_queries
   const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + sp.x;
   const int parts = min(kMergeWarps, K);
-  const OutRows out = out_rows(a, b, g);
+  const OutRowsT<kBf16> out = out_rows<kBf16>(a, b, g);
+#pragma unroll
   for (int qi = 0; qi < nq; ++qi) {   // a piece's record of query qi: slot * nq + qi
     if (warp < parts) {
       const int cnt = (K - warp + kMergeWarps - 1) / kMergeWarps;
       merge_partials<false>(a.partials + ((S0 + warp) * nq + qi) * kPartialFloats, cnt,
-                            kMergeWarps * nq, s_part[warp], nullptr, 0, lane);
+                            kMergeWarps * nq, s_part[warp],
+                            static_cast<const OutRowsT<kBf16>*>(nullptr), 0, lane);
     }
     __syncthreads();
     if (warp == 0) merge_partials<true>(&s_part[0][0], parts, 1, nullptr, &out, qi, lane);
-    __syncthreads();   // s_part is rewritten for the next query
+    if (qi + 1 < nq) __syncthreads();   // s_part is rewritten for the next query
   }
 }
 
@@ -1172,7 +1183,9 @@ cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, merge_kernel, a, static_cast<int32_t>(plan.grid));
+  auto merge = a.num_queries == 2 ? (a.out_bf16 ? merge_kernel<2, true> : merge_kernel<2, false>)
+                                  : (a.out_bf16 ? merge_kernel<1, true> : merge_kernel<1, false>);
+  return cudaLaunchKernelEx(&cfg, merge, a, static_cast<int32_t>(plan.grid));
 }
 
 }  // namespace pkv
