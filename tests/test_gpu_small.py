@@ -200,3 +200,23 @@ def test_bounded_wait_reports_timeout_and_context_survives(kernel):
     got = g.decode(kernel=kernel)
     assert pkv.get_device_error(g.pool) == 0
     assert max_err(got, g.oracle()) <= ATOL
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("grid,min_chunk", [(0, 0), (7, 0), (0, 3), (400, 0), (600, 1)])
+def test_stale_workspace_contents_do_not_matter(kernel, grid, min_chunk):
+    # The merge may only read partial records that this launch wrote: a
+    # workspace full of earlier records (here: NaN bytes, and then the
+    # records of a different batch) must give the same result.
+    c = make_case([300, 1, 47, 129, 16, 517, 2], seed=41, spare_pages=5)
+    g = GpuCase(c)
+    want = g.oracle(scale=0.11)
+    ws = g.pool.workspace(7, kernel, grid)
+    ws.fill_(0xFF)                       # every float of it is NaN
+    got = g.decode(scale=0.11, kernel=kernel, grid_ctas=grid, min_chunk=min_chunk, workspace=ws)
+    assert np.isfinite(got).all()
+    assert max_err(got, want) <= ATOL
+    other = GpuCase(make_case([900, 33, 400, 5, 260, 1, 1200], seed=42, spare_pages=2))
+    other.decode(kernel=kernel, grid_ctas=grid, min_chunk=min_chunk, workspace=ws)
+    again = g.decode(scale=0.11, kernel=kernel, grid_ctas=grid, min_chunk=min_chunk, workspace=ws)
+    assert np.array_equal(again, got)
