@@ -286,9 +286,17 @@ def run_ours(args, rank, world, local_rank):
     fused = not args.unfused and args.queries == 1
     out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
     r = Runner(w, device, kernel, fused, args.queries, out_dtype)
+    flags = 0
     if not args.no_pdl:
-        # no kernel of the step writes the lengths or the block tables
-        r.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES)
+        # No kernel of the step writes the lengths or the block tables.  With
+        # no separate append, the kernel before each decode (the previous
+        # layer's decode or merge) writes no page that decode reads, so its
+        # first page loads may start early too (--early-pages; measured: 2 %
+        # faster on llama1b_b16, no gain on the batch-64 mix).
+        flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES
+        if (fused or args.queries == 2) and args.early_pages:
+            flags |= pkv.LAUNCH_EARLY_PAGES
+        r.pool.set_launch_flags(flags)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -359,8 +367,9 @@ def run_ours(args, rank, world, local_rank):
             "launch": "one CUDA graph per step (16 x %s + split merge)%s" %
                       ("fused append+decode" if fused else
                        "two-query decode" if r.queries == 2 else "append + decode",
-                       "" if args.no_pdl else ", programmatic dependent launch, tables read "
-                                              "before the preceding kernel ends"),
+                       "" if args.no_pdl else ", programmatic dependent launch, tables %sread "
+                                              "before the preceding kernel ends" %
+                       ("and first pages " if flags & pkv.LAUNCH_EARLY_PAGES else "")),
             "l2": "inputs larger than L2: one step reads %.0f MB of K/V" %
                   (w.kv_bytes(1) * w.num_layers / 1e6),
         },
@@ -575,6 +584,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fill", action="store_true", help="skip the prefill fill timing")
+    ap.add_argument("--early-pages", action="store_true",
+                    help="start the first page loads before the preceding kernel ends")
     ap.add_argument("--queries", type=int, default=1, choices=[1, 2],
                     help="queries per sequence (2: causal pair, decode only)")
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])

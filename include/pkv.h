@@ -93,6 +93,8 @@ typedef enum {
 #define PKV_LAUNCH_PDL 1          /* programmatic dependent launch (see below) */
 #define PKV_LAUNCH_EARLY_TABLES 2 /* with PDL: decode reads seq_lens and block
                                      tables before the preceding kernel ends */
+#define PKV_LAUNCH_EARLY_PAGES 4  /* with PDL | EARLY_TABLES: decode also starts
+                                     its first page loads before then */
 #define PKV_LAUNCH_TEST_STALL (1 << 30) /* testing only: decode withholds one
                                      page so its bounded waits run out (~1 s)
                                      and it reports PKV_ERR_DEVICE_TIMEOUT */
@@ -139,12 +141,21 @@ PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
  * overlaps that kernel; the caller guarantees that the kernel launched just
  * before a decode does not write seq_lens or the block tables (an append,
  * which only reads them, is fine).
+ * PKV_LAUNCH_EARLY_PAGES (only together with both) lets decode also start
+ * loading the first pages of its range -- the KV of tokens already in the
+ * cache -- before that kernel has finished, so their memory latency overlaps
+ * it; q, the new token's rows and the outputs still wait.  The caller
+ * guarantees that the kernel launched just before a decode does not write
+ * the pool pages it reads: true when that kernel is the previous layer's
+ * decode or merge, or a projection that writes q; false when it is a
+ * pkv_append or pkv_fill into this layer (use the fused call instead).
  * PKV_LAUNCH_TEST_STALL exists only to test the device-timeout path: the
  * decode kernel never fills one shared-memory stage, every wait on it gives
  * up after about a second, the kernel exits early with garbage output and
  * pkv_get_device_error reports PKV_ERR_DEVICE_TIMEOUT; the context stays
  * usable.
- * flags: 0, PKV_LAUNCH_PDL or PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES,
+ * flags: 0, PKV_LAUNCH_PDL, PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES or
+ * PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES | PKV_LAUNCH_EARLY_PAGES,
  * optionally | PKV_LAUNCH_TEST_STALL, else PKV_ERR_INVALID_ARG.
  */
 PKV_API int pkv_pool_set_launch_flags(pkv_pool *pool, int32_t flags);

@@ -833,7 +833,11 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   // With kLaunchEarlyTables the lengths and block tables are read before the
   // preceding kernel of the stream has finished (the caller guarantees that
   // kernel does not write them); q, the pool and the outputs only after.
+  // With kLaunchEarlyPages as well, the first kS pages' loads are issued
+  // before that kernel has finished too (the caller guarantees it does not
+  // write those pages); their query rows and new-token rows only after.
   const bool early = (a.flags & kLaunchEarlyTables) != 0;
+  const bool early_pages = early && (a.flags & kLaunchEarlyPages) != 0;
   if (!early) pdl_wait();
   pdl_trigger();
   cta_lengths(a, s_len, s_pfx, reinterpret_cast<int32_t*>(smem + L::tot));
@@ -856,24 +860,26 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
     load_page_batch(a, s_pfx, p0 + lane, p0, p1, cur_phys, cur_info);
     load_page_batch(a, s_pfx, p0 + 32 + lane, p0, p1, nxt_phys, nxt_info);
   }
-  if (early) pdl_wait();
-
-  // empty (or invalid) sequences: zero output rows, once across the grid
-  for (int b = blockIdx.x * kWarps + warp; b < B; b += G * kWarps)
-    if (s_pfx[b + 1] == s_pfx[b]) zero_rows(a, b, lane);
-  if (n <= 0) return;
-  // Issue page r into stage r % kS (warp 0 only; stage known to be free).
+  // Issue page r into stage r % kS (warp 0 only; stage known to be free):
+  // kIssuePage arms the stage's full barrier with all its bytes and starts
+  // the page's TMA load; kIssueRows starts the bulk copies of the query rows
+  // (first page of a sequence in this range) and of the new token's rows
+  // (fused append, last page of a sequence).  A first-batch page (r < 32)
+  // may take the two parts at different times.
   // Test-only: leave page 0's full barrier unarmed, so the consumers' bounded
   // waits run out and the launch reports PKV_ERR_DEVICE_TIMEOUT.
+  constexpr int kIssuePage = 1, kIssueRows = 2;
   const bool stall = (a.flags & kLaunchTestStall) != 0;
   int issued = 0;   // pages issued so far (warp 0)
-  auto issue = [&](int r) {
-    ++issued;
-    if ((r >> 5) != cur_k) {
-      cur_phys = nxt_phys;
-      cur_info = nxt_info;
-      ++cur_k;
-      load_page_batch(a, s_pfx, p0 + 32 * (cur_k + 1) + lane, p0, p1, nxt_phys, nxt_info);
+  auto issue = [&](int r, int part) {
+    if (part & kIssuePage) {
+      ++issued;
+      if ((r >> 5) != cur_k) {
+        cur_phys = nxt_phys;
+        cur_info = nxt_info;
+        ++cur_k;
+        load_page_batch(a, s_pfx, p0 + 32 * (cur_k + 1) + lane, p0, p1, nxt_phys, nxt_info);
+      }
     }
     const int32_t phys = __shfl_sync(kFull, cur_phys, r & 31);
     const int32_t info = __shfl_sync(kFull, cur_info, r & 31);
@@ -885,14 +891,20 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
       const bool start = info & 1;
       const bool append = fused && (info & 2);
       const int64_t seq = info >> 2;
-      s_flags[st] = ok ? 0 : 1;
-      s_phys[st] = phys;
-      if (!ok) record_error(a.err, kErrBadPage);
-      const uint32_t bytes =
-          (ok ? kPageBytes : 0) + (start ? nq * kQRowsBytes : 0) + (append ? kNewRowsBytes : 0);
-      if (bytes) {
-        mbar_arrive_expect_tx(bar, bytes);
-        if (ok) tma_load_tile(dst, &tmap, 0, phys * kRowsPerPage, bar, policy);
+      const uint32_t rows = (start ? nq * kQRowsBytes : 0) + (append ? kNewRowsBytes : 0);
+      if (part & kIssuePage) {
+        s_flags[st] = ok ? 0 : 1;
+        s_phys[st] = phys;
+        if (!ok) record_error(a.err, kErrBadPage);
+        const uint32_t bytes = (ok ? kPageBytes : 0) + rows;
+        if (bytes) {
+          mbar_arrive_expect_tx(bar, bytes);
+          if (ok) tma_load_tile(dst, &tmap, 0, phys * kRowsPerPage, bar, policy);
+        } else {
+          mbar_arrive(bar);
+        }
+      }
+      if (part & kIssueRows) {
         if (start)
           bulk_load(dst + kPageBytes, a.q + seq * nq * kQHeads * kDim, nq * kQRowsBytes, bar);
         if (append) {
@@ -901,13 +913,20 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
           bulk_load(nd + kNewRowsBytes / 2, a.v_new + seq * kKvHeads * kDim, kNewRowsBytes / 2,
                     bar);
         }
-      } else {
-        mbar_arrive(bar);
       }
     }
   };
+  if (warp == 0 && early_pages)
+    for (int r = 0; r < n && r < kS; ++r) issue(r, kIssuePage);
+  if (early) pdl_wait();
+
+  // empty (or invalid) sequences: zero output rows, once across the grid
+  for (int b = blockIdx.x * kWarps + warp; b < B; b += G * kWarps)
+    if (s_pfx[b + 1] == s_pfx[b]) zero_rows(a, b, lane);
+  if (n <= 0) return;
   if (warp == 0)
-    for (int r = 0; r < n && r < kS; ++r) issue(r);
+    for (int r = 0; r < n && r < kS; ++r)
+      issue(r, early_pages ? kIssueRows : kIssuePage | kIssueRows);
   // After a timed-out wait: wait (bounded) for the copies still in flight
   // into this CTA's stages, pages k0 .. issued-1, before the CTA exits.
   auto drain = [&](int k0) {
@@ -939,7 +958,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
         drain(r);
         return;
       }
-      issue(rr + kS);
+      issue(rr + kS, kIssuePage | kIssueRows);
     }
     const uint32_t fb = full + 8 * st;
     const uint32_t par = static_cast<uint32_t>(r / kS) & 1u;

@@ -204,9 +204,12 @@ int pkv_fill(pkv_pool* pool, const int32_t* block_tables, const int32_t* cu_toke
 }
 
 int pkv_pool_set_launch_flags(pkv_pool* pool, int32_t flags) {
-  if (!pool || (flags & ~(PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES | PKV_LAUNCH_TEST_STALL)))
+  if (!pool || (flags & ~(PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES | PKV_LAUNCH_EARLY_PAGES |
+                          PKV_LAUNCH_TEST_STALL)))
     return PKV_ERR_INVALID_ARG;
   if ((flags & PKV_LAUNCH_EARLY_TABLES) && !(flags & PKV_LAUNCH_PDL)) return PKV_ERR_INVALID_ARG;
+  if ((flags & PKV_LAUNCH_EARLY_PAGES) && !(flags & PKV_LAUNCH_EARLY_TABLES))
+    return PKV_ERR_INVALID_ARG;
   pool->launch_flags = flags;
   return PKV_OK;
 }

@@ -202,6 +202,7 @@ constexpr int kSeqCost = 1;
 // Launch flags (pool-wide).
 constexpr int kLaunchPdl = 1;         // programmatic dependent launch
 constexpr int kLaunchEarlyTables = 2; // read seq_lens / block tables before waiting
+constexpr int kLaunchEarlyPages = PKV_LAUNCH_EARLY_PAGES;  // + first page loads too
 constexpr int kLaunchTestStall = PKV_LAUNCH_TEST_STALL;  // testing the timeout path only
 
 struct DecodeArgs {

@@ -28,6 +28,7 @@ DTYPE_F32, DTYPE_BF16 = 0, 1
 MAX_QUERIES = 2
 LAUNCH_PDL = 1
 LAUNCH_EARLY_TABLES = 2
+LAUNCH_EARLY_PAGES = 4
 LAUNCH_TEST_STALL = 1 << 30
 
 OK = 0

@@ -90,13 +90,18 @@ def test_fused_split_patterns_bitwise_equal_to_two_calls(kernel, grid, min_chunk
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_fused_repeated_steps_with_pdl(kernel):
-    # several decode steps: lengths grow by one, each step appends and attends
+@pytest.mark.parametrize("flags", [pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES,
+                                   pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES |
+                                   pkv.LAUNCH_EARLY_PAGES])
+def test_fused_repeated_steps_with_pdl(kernel, flags):
+    # several decode steps: lengths grow by one, each step appends and attends;
+    # with early pages each launch starts loading its first pages while the
+    # previous step's kernels run (they write other slots only)
     lens0 = np.array([40, 1, 77, 15, 300], np.int32)
     steps = 20
     c = make_case(list(lens0 + steps), seed=31, spare_pages=3)
     g = GpuCase(c)
-    g.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES)
+    g.pool.set_launch_flags(flags)
     host = c["pool"].copy()
     rng = np.random.default_rng(5)
     from tests.cases import bf16_bits
