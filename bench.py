@@ -213,8 +213,9 @@ class Runner:
         # one set of per-layer inputs, reused every step (values do not change timing)
         ins = [W.step_inputs(w, 1, l, device) for l in range(nl)]
         self.q = torch.stack([x[0] for x in ins])
-        if queries == 2:   # a second query per sequence: the first one again, shifted in value
-            self.q = torch.stack([self.q, (self.q.float() * 0.5).to(torch.bfloat16)], dim=2)
+        if queries > 1:   # more queries per sequence: the first one again, scaled
+            self.q = torch.stack([(self.q.float() * (1.0 - 0.1 * i)).to(torch.bfloat16)
+                                  for i in range(queries)], dim=2)
         self.k = torch.stack([x[1] for x in ins])
         self.v = torch.stack([x[2] for x in ins])
         oshape = (nl, B, 32, 64) if queries == 1 else (nl, B, queries, 32, 64)
@@ -241,7 +242,7 @@ class Runner:
         pkv = self.pkv
         sl = self.seq_lens[variant]
         for l in range(self.w.num_layers):
-            if self.queries == 2 or self.out_dtype != torch.float32:
+            if self.queries > 1 or self.out_dtype != torch.float32:
                 kv = dict(k_new=self.k[l], v_new=self.v[l]) if self.fused else {}
                 if not self.fused and not decode_only and self.queries == 1:
                     pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
@@ -307,7 +308,7 @@ def run_ours(args, rank, world, local_rank):
         # first page loads may start early too (--early-pages; measured: 2 %
         # faster on llama1b_b16, no gain on the batch-64 mix).
         flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES
-        if (fused or args.queries == 2) and args.early_pages:
+        if (fused or args.queries > 1) and args.early_pages:
             flags |= pkv.LAUNCH_EARLY_PAGES
         r.pool.set_launch_flags(flags)
     stream = torch.cuda.Stream(device)
@@ -379,7 +380,7 @@ def run_ours(args, rank, world, local_rank):
             "queries_per_sequence": r.queries, "out_dtype": args.out_dtype,
             "launch": "one CUDA graph per step (16 x %s + split merge)%s" %
                       ("fused append+decode" if fused else
-                       "two-query decode" if r.queries == 2 else "append + decode",
+                       "%d-query decode" % r.queries if r.queries > 1 else "append + decode",
                        "" if args.no_pdl else ", programmatic dependent launch, tables %sread "
                                               "before the preceding kernel ends" %
                        ("and first pages " if flags & pkv.LAUNCH_EARLY_PAGES else "")),
@@ -397,7 +398,7 @@ def run_ours(args, rank, world, local_rank):
         "decode_queries_per_s": w.batch * r.queries / avg_dec_s,
         "e2e": e2e,
         "prefill_fill": fill,
-        "gpu_launches": (args.steps * w.num_layers * (2 if fused or r.queries == 2 else 3) +
+        "gpu_launches": (args.steps * w.num_layers * (2 if fused or r.queries > 1 else 3) +
                          (0 if fused else dec_launches * 2)),
         "decode_timing": ("CUDA events around the %d full-step replays (fused append + decode "
                           "+ merge per layer, %d launches)" % (args.steps, dec_launches)
@@ -626,8 +627,8 @@ def main():
     ap.add_argument("--no-fill", action="store_true", help="skip the prefill fill timing")
     ap.add_argument("--early-pages", action="store_true",
                     help="start the first page loads before the preceding kernel ends")
-    ap.add_argument("--queries", type=int, default=1, choices=[1, 2],
-                    help="queries per sequence (2: causal pair, decode only)")
+    ap.add_argument("--queries", type=int, default=1, choices=range(1, 9),
+                    help="queries per sequence (> 1: causal among them, decode only)")
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])
     ap.add_argument("--unfused", action="store_true",
                     help="separate append and decode launches instead of the fused call")

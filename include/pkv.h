@@ -302,13 +302,14 @@ PKV_API int paged_attention_decode_append_ex(const uint16_t *q, const uint16_t *
  * lack, in one parameter block (future fields are appended; struct_size
  * tells the library which fields the caller knows).
  *
- *  - num_queries = 2: two queries per sequence, causal between them (the
- *    plainest multi-token decode, as in checking a drafted token): q and out
- *    are [batch][2][32][64]; query i of sequence b attends to tokens
- *    t < seq_lens[b] - 1 + i, i.e. query 0 does not see the last token.
- *    Needs seq_lens[b] = 0 or >= 2 (1 -> PKV_ERR_BAD_SEQ_LEN, zero rows),
- *    the tensor-core kernel (PKV_KERNEL_SIMT -> PKV_ERR_UNSUPPORTED) and no
- *    fused append (k_new must be NULL: write the two tokens with pkv_fill).
+ *  - num_queries = T in 2..8: T queries per sequence, causal among them
+ *    (the plainest multi-token decode, as in checking T - 1 drafted tokens):
+ *    q and out are [batch][T][32][64]; query i of sequence b attends to
+ *    tokens t < seq_lens[b] - T + 1 + i, so query T-1 sees the whole context
+ *    and each earlier query one token fewer.  Needs seq_lens[b] = 0 or >= T
+ *    (1..T-1 -> PKV_ERR_BAD_SEQ_LEN, zero rows), the tensor-core kernel
+ *    (PKV_KERNEL_SIMT -> PKV_ERR_UNSUPPORTED) and no fused append (k_new must
+ *    be NULL: write the T tokens with pkv_fill).
  *  - out_dtype = PKV_DTYPE_BF16: the output rows are BF16, rounded to
  *    nearest even from the FP32 result (the pages warn that BF16 rounding
  *    can differ with the batch size: "Curso gratuito recorre la inferencia
@@ -340,7 +341,7 @@ typedef struct pkv_decode_params {
   int32_t num_layers;
   int32_t batch;
   int32_t max_blocks;
-  int32_t num_queries; /* 1 or 2 */
+  int32_t num_queries; /* 1..8 */
   int32_t out_dtype;   /* PKV_DTYPE_F32 or PKV_DTYPE_BF16 */
   int32_t kernel;
   int32_t grid_ctas;

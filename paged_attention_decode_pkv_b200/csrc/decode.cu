@@ -72,7 +72,6 @@ struct StageLayout {
   static constexpr int kBytes = kPageBytes + kQBytes + kNewRowsBytes;
   static_assert(kBytes % 1024 == 0, "stage alignment");
 };
-constexpr int kScratchBytes = 512;                  // per-warp P^T transpose buffer
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -135,7 +134,8 @@ struct OutRowsT {
 struct SimtCompute {
   static constexpr int kStages = 3;
   static constexpr int kMinBlocks = 1;
-  static constexpr int kQueries = 1;
+  static constexpr int kMaxQueries = 1;
+  static constexpr int kScratch = 512;
 
   float2 q2[kGroup][4];   // q[h][8c + 2e], q[h][8c + 2e + 1]
   float2 acc[kGroup][4];  // sum over this lane's tokens of p * v[8c + 2e ..]
@@ -161,8 +161,8 @@ struct SimtCompute {
   }
 
   __device__ __forceinline__ void consume(uint32_t ktile, uint32_t vtile, uint32_t /*scratch*/,
-                                          int nvalid, int /*nvalid_q0*/, float scale_log2,
-                                          int lane) {
+                                          int rem, float scale_log2, int lane) {
+    const int nvalid = min(kTokens, rem);
     const int c = lane & 7, tg = lane >> 3;
     const int b0 = c & 1, b1 = (c >> 1) & 1, b2 = c >> 2;
 
@@ -353,99 +353,119 @@ struct SimtCompute {
 //  Lane holds O^T[16mt + r (+8)][2qd..2qd+1]: its softmax heads and its
 //  accumulator heads are the same, so rescaling needs no data movement.
 // ---------------------------------------------------------------------------
-template <int kNq>   // queries per sequence: 1, or 2 in the zero columns
+// kNt n-tiles of the MMA's N = 8: column n of tile nt is head n % 4 of
+// query 2 nt + n / 4, so one K/V stream serves up to 2 kNt queries of a
+// sequence.  kOne: exactly one query (tile 0's columns 4..7 stay zero); its
+// masks and guards are then compile-time.
+template <int kNt, bool kOne>
 struct MmaComputeT {
   static constexpr int kStages = 2;
-  static constexpr int kMinBlocks = 2;
-  static constexpr int kQueries = kNq;
+  static constexpr int kMinBlocks = kNt == 1 ? 2 : 1;
+  static constexpr int kMaxQueries = kOne ? 1 : 2 * kNt;
+  static constexpr int kScratch = kNt * 512;   // per-warp P^T transpose buffers
 
-  uint32_t qb[4][2];  // B fragments of Q^T, k-steps 0..3 (zero for lanes with r >= 4)
-  float o[4][4];      // O^T accumulators, m-tiles 0..3
-  float m[2];         // running max of heads 2qd, 2qd+1 (log2 units)
-  float l[2];         // this lane's share of the softmax denominators
+  uint32_t qb[kNt][4][2];  // B fragments of Q^T, k-steps 0..3 (zero for absent queries)
+  float o[kNt][4][4];      // O^T accumulators, m-tiles 0..3
+  float m[kNt][2];         // running max of the lane's two columns (log2 units)
+  float l[kNt][2];         // this lane's share of the softmax denominators
+  int nq;                  // queries of the sequence
 
-  // qrows: the staged query rows ([query][32 heads][64]); column n of the
-  // MMA's N = 8 is head n % 4 of query n / 4 (the columns of a second query
-  // stay zero when there is one).
-  __device__ __forceinline__ void begin(uint32_t qrows, int warp, int /*nq*/, int lane) {
+  // qrows: the staged query rows ([query][32 heads][64]).
+  __device__ __forceinline__ void begin(uint32_t qrows, int warp, int nq_, int lane) {
+    nq = kOne ? 1 : nq_;
     const int r = lane >> 2, qd = lane & 3;
-    const int qi = r / kGroup;
-    constexpr int nq = kNq;
-    const uint32_t row = qrows + (qi * kQHeads + warp * kGroup + r % kGroup) * kRowBytes;
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      if (qi < nq) {
-        const uint32_t a = row + (16 * ks + 2 * qd) * 2;
-        qb[ks][0] = lds32(a);
-        qb[ks][1] = lds32(a + 16);
-      } else {
-        qb[ks][0] = qb[ks][1] = 0u;
+    for (int nt = 0; nt < kNt; ++nt) {
+      const int qi = 2 * nt + r / kGroup;
+      const uint32_t row = qrows + (qi * kQHeads + warp * kGroup + r % kGroup) * kRowBytes;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        if (qi < nq) {
+          const uint32_t a = row + (16 * ks + 2 * qd) * 2;
+          qb[nt][ks][0] = lds32(a);
+          qb[nt][ks][1] = lds32(a + 16);
+        } else {
+          qb[nt][ks][0] = qb[nt][ks][1] = 0u;
+        }
       }
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[nt][mt][i] = 0.f;
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
     }
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
-    m[0] = m[1] = -INFINITY;
-    l[0] = l[1] = 0.f;
   }
 
-  // nvalid: tokens of this page in the context of the last query; nvalid_q0:
-  // in the context of query 0 of two (one fewer at the end; may be 0).
+  // rem: tokens from this page's first slot to the end of the context (of the
+  // last query); query q of nq sees nq - 1 - q tokens fewer, possibly none
+  // of this page.
   __device__ __forceinline__ void consume(uint32_t ktile, uint32_t vtile, uint32_t scratch,
-                                          int nvalid, int nvalid_q0, float scale_log2, int lane) {
+                                          int rem, float scale_log2, int lane) {
     const int r = lane >> 2, qd = lane & 3;
-    // ---- S^T = K Q^T
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    const int nvalid = min(kTokens, rem);
+    // ---- S^T = K Q^T, each K fragment used by every n-tile
+    float s[kNt][4];
+#pragma unroll
+    for (int nt = 0; nt < kNt; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       uint32_t a[4];
       ldsm_x4(a, ktile + swz(lane & 15, 2 * ks + (lane >> 4)));
-      mma_bf16_16816(s, a, qb[ks][0], qb[ks][1]);
-    }
-    // ---- FP32 online softmax; tokens r and r + 8, columns 2qd and 2qd + 1
-    // (query qd / 2)
-    const int nv = (kNq == 2 && qd < 2) ? nvalid_q0 : nvalid;
-    const bool v0 = r < nv, v1 = r + 8 < nv;
-    const float x0 = v0 ? s[0] * scale_log2 : -INFINITY;
-    const float x1 = v0 ? s[1] * scale_log2 : -INFINITY;
-    const float x2 = v1 ? s[2] * scale_log2 : -INFINITY;
-    const float x3 = v1 ? s[3] * scale_log2 : -INFINITY;
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+      for (int nt = 0; nt < kNt; ++nt) mma_bf16_16816(s[nt], a, qb[nt][ks][0], qb[nt][ks][1]);
     }
-    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-    // a column with no valid score yet (query 0's context can end a page
-    // early) keeps m = -inf: subtract 0 there, so that -inf - -inf never
-    // appears; its p and the rescale factor are then 0
-    const float r0 = (kNq == 2 && mn0 == -INFINITY) ? 0.f : mn0;
-    const float r1 = (kNq == 2 && mn1 == -INFINITY) ? 0.f : mn1;
-    const float a0 = fast_exp2(m[0] - r0), a1 = fast_exp2(m[1] - r1);
-    m[0] = mn0;
-    m[1] = mn1;
-    const float p0 = fast_exp2(x0 - r0), p1 = fast_exp2(x1 - r1);
-    const float p2 = fast_exp2(x2 - r0), p3 = fast_exp2(x3 - r1);
-    l[0] = fmaf(l[0], a0, p0 + p2);
-    l[1] = fmaf(l[1], a1, p1 + p3);
-    // ---- P^T, split into BF16 hi + lo, through the scratch ([t][8 heads])
-    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
-    const uint32_t l01 = pack_bf16x2(p0 - __uint_as_float(h01 << 16),
-                                     p1 - __uint_as_float(h01 & 0xFFFF0000u));
-    const uint32_t l23 = pack_bf16x2(p2 - __uint_as_float(h23 << 16),
-                                     p3 - __uint_as_float(h23 & 0xFFFF0000u));
-    __syncwarp();   // previous tile's scratch reads are done
-    const uint32_t w0 = scratch + r * 16 + qd * 4;
-    sts32(w0, h01);
-    sts32(w0 + 128, h23);
-    sts32(w0 + 256, l01);
-    sts32(w0 + 384, l23);
+    uint32_t pb[kNt][4];   // per tile: hi b0, b1; lo b0, b1
+    float a0[kNt], a1[kNt];
+#pragma unroll
+    for (int nt = 0; nt < kNt; ++nt) {
+      // ---- FP32 online softmax; tokens r and r + 8, columns 2qd and 2qd + 1
+      // (query 2 nt + qd / 2)
+      const int nv = kOne ? nvalid : min(kTokens, rem - (nq - 1 - (2 * nt + (qd >> 1))));
+      const bool v0 = r < nv, v1 = r + 8 < nv;
+      const float x0 = v0 ? s[nt][0] * scale_log2 : -INFINITY;
+      const float x1 = v0 ? s[nt][1] * scale_log2 : -INFINITY;
+      const float x2 = v1 ? s[nt][2] * scale_log2 : -INFINITY;
+      const float x3 = v1 ? s[nt][3] * scale_log2 : -INFINITY;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+      }
+      const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+      // a column with no valid score yet (an earlier query's context can end
+      // a page early) keeps m = -inf: subtract 0 there, so that -inf - -inf
+      // never appears; its p and the rescale factor are then 0
+      const float r0 = (!kOne && mn0 == -INFINITY) ? 0.f : mn0;
+      const float r1 = (!kOne && mn1 == -INFINITY) ? 0.f : mn1;
+      a0[nt] = fast_exp2(m[nt][0] - r0);
+      a1[nt] = fast_exp2(m[nt][1] - r1);
+      m[nt][0] = mn0;
+      m[nt][1] = mn1;
+      const float p0 = fast_exp2(x0 - r0), p1 = fast_exp2(x1 - r1);
+      const float p2 = fast_exp2(x2 - r0), p3 = fast_exp2(x3 - r1);
+      l[nt][0] = fmaf(l[nt][0], a0[nt], p0 + p2);
+      l[nt][1] = fmaf(l[nt][1], a1[nt], p1 + p3);
+      // ---- P^T, split into BF16 hi + lo, through the tile's scratch ([t][8])
+      const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+      const uint32_t l01 = pack_bf16x2(p0 - __uint_as_float(h01 << 16),
+                                       p1 - __uint_as_float(h01 & 0xFFFF0000u));
+      const uint32_t l23 = pack_bf16x2(p2 - __uint_as_float(h23 << 16),
+                                       p3 - __uint_as_float(h23 & 0xFFFF0000u));
+      const uint32_t sc = scratch + nt * 512;
+      if (nt == 0) __syncwarp();   // previous page's scratch reads are done
+      const uint32_t w0 = sc + r * 16 + qd * 4;
+      sts32(w0, h01);
+      sts32(w0 + 128, h23);
+      sts32(w0 + 256, l01);
+      sts32(w0 + 384, l23);
+    }
     __syncwarp();
-    uint32_t pb[4];   // hi: b0, b1; lo: b0, b1
-    ldsm_x4_trans(pb, scratch + (lane >> 3) * 128 + (lane & 7) * 16);
-    // ---- rescale and O^T += V^T P^T (hi, lo)
+#pragma unroll
+    for (int nt = 0; nt < kNt; ++nt)
+      ldsm_x4_trans(pb[nt], scratch + nt * 512 + (lane >> 3) * 128 + (lane & 7) * 16);
+    // ---- rescale and O^T += V^T P^T (hi, lo), each V fragment used by every tile
     uint32_t mlo = kFull, mhi = kFull;
     if (nvalid < kTokens) {   // zero V rows past the context: 0 * NaN would be NaN
       const int t = 2 * qd;
@@ -462,19 +482,22 @@ struct MmaComputeT {
       a[1] &= mlo;
       a[2] &= mhi;
       a[3] &= mhi;
-      o[mt][0] *= a0;
-      o[mt][1] *= a1;
-      o[mt][2] *= a0;
-      o[mt][3] *= a1;
-      mma_bf16_16816(o[mt], a, pb[0], pb[1]);
-      mma_bf16_16816(o[mt], a, pb[2], pb[3]);
+#pragma unroll
+      for (int nt = 0; nt < kNt; ++nt) {
+        o[nt][mt][0] *= a0[nt];
+        o[nt][mt][1] *= a1[nt];
+        o[nt][mt][2] *= a0[nt];
+        o[nt][mt][3] *= a1[nt];
+        mma_bf16_16816(o[nt][mt], a, pb[nt][0], pb[nt][1]);
+        mma_bf16_16816(o[nt][mt], a, pb[nt][2], pb[nt][3]);
+      }
     }
   }
 
-  // Full softmax denominators of heads 2qd, 2qd + 1.
-  __device__ __forceinline__ void reduce_l(float& l0, float& l1) const {
-    l0 = l[0];
-    l1 = l[1];
+  // Full softmax denominators of tile nt's columns 2qd, 2qd + 1.
+  __device__ __forceinline__ void reduce_l(int nt, float& l0, float& l1) const {
+    l0 = l[nt][0];
+    l1 = l[nt][1];
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       l0 += __shfl_xor_sync(kFull, l0, off);
@@ -482,47 +505,51 @@ struct MmaComputeT {
     }
   }
 
-  // O^T columns 2qd, 2qd + 1 = query qd / 2, heads 2(qd % 2), 2(qd % 2) + 1,
-  // scaled by s0, s1; lanes whose query does not exist write nothing.
+  // Tile nt's O^T columns 2qd, 2qd + 1 = query 2 nt + qd / 2, heads
+  // 2(qd % 2) and 2(qd % 2) + 1, scaled by s0, s1; absent queries write nothing.
   template <class Out>
-  __device__ __forceinline__ void write_rows(const Out& out, int lane, float s0,
+  __device__ __forceinline__ void write_rows(const Out& out, int nt, int lane, float s0,
                                              float s1) const {
-    constexpr int nq = kNq;
     const int r = lane >> 2, qd = lane & 3;
-    const int qi = qd >> 1, h = 2 * (qd & 1);
+    const int qi = 2 * nt + (qd >> 1), h = 2 * (qd & 1);
     if (qi < nq) {
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
-        out.put(qi, h, 16 * mt + r, o[mt][0] * s0);
-        out.put(qi, h + 1, 16 * mt + r, o[mt][1] * s1);
-        out.put(qi, h, 16 * mt + r + 8, o[mt][2] * s0);
-        out.put(qi, h + 1, 16 * mt + r + 8, o[mt][3] * s1);
+        out.put(qi, h, 16 * mt + r, o[nt][mt][0] * s0);
+        out.put(qi, h + 1, 16 * mt + r, o[nt][mt][1] * s1);
+        out.put(qi, h, 16 * mt + r + 8, o[nt][mt][2] * s0);
+        out.put(qi, h + 1, 16 * mt + r + 8, o[nt][mt][3] * s1);
       }
     }
   }
 
   template <class Out>
   __device__ __forceinline__ void finalize(const Out& out, int lane) const {
-    float l0, l1;
-    reduce_l(l0, l1);
-    write_rows(out, lane, 1.f / l0, 1.f / l1);
+#pragma unroll
+    for (int nt = 0; nt < kNt; ++nt) {
+      float l0, l1;
+      reduce_l(nt, l0, l1);
+      write_rows(out, nt, lane, 1.f / l0, 1.f / l1);
+    }
   }
 
   // Partial records, one per query: P + i * kPartialFloats = m[4], l[4],
   // acc[4][64] of query i (unnormalised).
   __device__ __forceinline__ void store_partial(float* P, int /*nq*/, int lane) const {
-    constexpr int nq = kNq;
-    float l0, l1;
-    reduce_l(l0, l1);
-    const int qd = lane & 3, qi = qd >> 1, h = 2 * (qd & 1);
-    if (lane < 4 && qi < nq) {   // r == 0
-      float* rec = P + qi * kPartialFloats;
-      rec[h] = m[0];
-      rec[h + 1] = m[1];
-      rec[kGroup + h] = l0;
-      rec[kGroup + h + 1] = l1;
+#pragma unroll
+    for (int nt = 0; nt < kNt; ++nt) {
+      float l0, l1;
+      reduce_l(nt, l0, l1);
+      const int qd = lane & 3, qi = 2 * nt + (qd >> 1), h = 2 * (qd & 1);
+      if (lane < 4 && qi < nq) {   // r == 0
+        float* rec = P + qi * kPartialFloats;
+        rec[h] = m[nt][0];
+        rec[h + 1] = m[nt][1];
+        rec[kGroup + h] = l0;
+        rec[kGroup + h + 1] = l1;
+      }
+      write_rows(OutRowsT<false>{P + 2 * kGroup, kPartialFloats}, nt, lane, 1.f, 1.f);
     }
-    write_rows(OutRowsT<false>{P + 2 * kGroup, kPartialFloats}, lane, 1.f, 1.f);
   }
 };
 
@@ -786,9 +813,9 @@ template <class C>
 struct SmemPlan {
   static constexpr int S = C::kStages;
   static constexpr size_t stages = 0;   // [S][page 32 KiB | query rows 4 KiB]
-  static constexpr int kStageBytes = StageLayout<C::kQueries>::kBytes;
+  static constexpr int kStageBytes = StageLayout<C::kMaxQueries>::kBytes;
   static constexpr size_t scratch = stages + size_t(S) * kStageBytes;
-  static constexpr size_t full = scratch + size_t(kWarps) * kScratchBytes;
+  static constexpr size_t full = scratch + size_t(kWarps) * C::kScratch;
   static constexpr size_t empty = full + size_t(S) * 8;
   static constexpr size_t flags = empty + size_t(S) * 8;   // [S] bad page, [1] abort
   static constexpr size_t phys = flags + size_t(S + 1) * 4;  // [S] physical page of the stage
@@ -813,12 +840,12 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   volatile int32_t* s_flags = reinterpret_cast<int32_t*>(smem + L::flags);
   volatile int32_t* s_phys = reinterpret_cast<int32_t*>(smem + L::phys);
   const bool fused = a.k_new != nullptr;
-  constexpr int nq = C::kQueries;   // == a.num_queries (the host picks the variant)
+  const int nq = a.num_queries;   // <= C::kMaxQueries (the host picks the variant)
   int32_t* s_len = reinterpret_cast<int32_t*>(smem + L::lens);
   int32_t* s_pfx = s_len + B;
   const uint32_t base = smem_addr(smem);
   const uint32_t full = base + L::full, empty = base + L::empty;
-  const uint32_t scratch = base + L::scratch + warp * kScratchBytes;
+  const uint32_t scratch = base + L::scratch + warp * C::kScratch;
 
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -997,13 +1024,10 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
       __syncwarp();
     }
     if (!s_flags[st]) {
-      // tokens of this page in the context of the last query, and of the
-      // first of two (whose context ends one token earlier)
-      const int nvalid = min(kTokens, Lb - kTokens * j);
-      const int nvalid_q0 = nq == 1 ? nvalid : min(kTokens, Lb - 1 - kTokens * j);
+      // tokens from this page's first slot to the end of the (last query's) context
+      const int rem = Lb - kTokens * j;
       const uint32_t ktile = stage + warp * kTileBytes;
-      cmp.consume(ktile, ktile + kKvHeads * kTileBytes, scratch, nvalid, nvalid_q0, a.scale_log2,
-                  lane);
+      cmp.consume(ktile, ktile + kKvHeads * kTileBytes, scratch, rem, a.scale_log2, lane);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + 8 * st);
@@ -1036,7 +1060,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
 // ---------------------------------------------------------------------------
 constexpr int kMergeWarps = 8;
 
-template <int kNq, bool kBf16>
+template <int kNq, bool kBf16>   // kNq: queries per sequence, 0 = read from the arguments
 __global__ void __launch_bounds__(kMergeWarps * 32)
     merge_kernel(const DecodeArgs a, int32_t decode_grid) {
   __shared__ __align__(16) float s_part[kMergeWarps][kPartialFloats];
@@ -1081,7 +1105,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   if (K <= 1 && (g | b) != 0) return;
   pdl_wait();   // the pieces are written by the decode grid
   if (K <= 1) return;
-  constexpr int nq = kNq;   // == a.num_queries
+  const int nq = kNq > 0 ? kNq : a.num_queries;   // kNq == 0: any count
   const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + sp.x;
   const int parts = min(kMergeWarps, K);
   const OutRowsT<kBf16> out = out_rows<kBf16>(a, b, g);
@@ -1106,19 +1130,42 @@ static const void* kernel_ptr() {
   return reinterpret_cast<const void*>(&decode_kernel<C>);
 }
 
-using MmaCompute1 = MmaComputeT<1>;
-using MmaCompute2 = MmaComputeT<2>;
+// Tensor-core variants by queries per sequence: 1 (its own, fastest),
+// 2 (one n-tile), 3-4, 5-6, 7-8 (two to four n-tiles).
+using MmaQ1 = MmaComputeT<1, true>;
+using MmaQ2 = MmaComputeT<1, false>;
+using MmaQ4 = MmaComputeT<2, false>;
+using MmaQ6 = MmaComputeT<3, false>;
+using MmaQ8 = MmaComputeT<4, false>;
+
+// Calls f with a value of the compute type that serves (kernel, nq); false
+// if there is none.
+template <class F>
+static bool with_compute(int kernel, int nq, F&& f) {
+  if (kernel == PKV_KERNEL_SIMT) {
+    if (nq != 1) return false;
+    f(SimtCompute{});
+    return true;
+  }
+  if (kernel != PKV_KERNEL_MMA || nq < 1 || nq > kMaxQueries) return false;
+  if (nq == 1) f(MmaQ1{});
+  else if (nq == 2) f(MmaQ2{});
+  else if (nq <= 4) f(MmaQ4{});
+  else if (nq <= 6) f(MmaQ6{});
+  else f(MmaQ8{});
+  return true;
+}
 
 static const void* kernel_for(int kernel, int nq) {
-  if (kernel == PKV_KERNEL_SIMT) return nq == 1 ? kernel_ptr<SimtCompute>() : nullptr;
-  if (kernel == PKV_KERNEL_MMA)
-    return nq == 1 ? kernel_ptr<MmaCompute1>() : nq == 2 ? kernel_ptr<MmaCompute2>() : nullptr;
-  return nullptr;
+  const void* fn = nullptr;
+  with_compute(kernel, nq, [&](auto c) { fn = kernel_ptr<decltype(c)>(); });
+  return fn;
 }
 
 static size_t smem_for(int kernel, int nq, int32_t batch) {
-  if (kernel == PKV_KERNEL_SIMT) return SmemPlan<SimtCompute>::bytes(batch);
-  return nq == 2 ? SmemPlan<MmaCompute2>::bytes(batch) : SmemPlan<MmaCompute1>::bytes(batch);
+  size_t bytes = 0;
+  with_compute(kernel, nq, [&](auto c) { bytes = SmemPlan<decltype(c)>::bytes(batch); });
+  return bytes;
 }
 
 cudaError_t prepare_decode_kernels(int device) {
@@ -1126,7 +1173,8 @@ cudaError_t prepare_decode_kernels(int device) {
   cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
   if (e != cudaSuccess) return e;
   for (const void* fn : {kernel_for(PKV_KERNEL_SIMT, 1), kernel_for(PKV_KERNEL_MMA, 1),
-                          kernel_for(PKV_KERNEL_MMA, 2)}) {
+                          kernel_for(PKV_KERNEL_MMA, 2), kernel_for(PKV_KERNEL_MMA, 4),
+                          kernel_for(PKV_KERNEL_MMA, 6), kernel_for(PKV_KERNEL_MMA, 8)}) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, fn);
     if (e != cudaSuccess) return e;
@@ -1183,15 +1231,9 @@ static cudaError_t launch_one(const DecodePlan& plan, const CUtensorMap& tmap, c
 
 cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const DecodeArgs& a,
                           int flags, cudaStream_t stream) {
-  cudaError_t e;
-  switch (plan.kernel) {
-    case PKV_KERNEL_SIMT: e = launch_one<SimtCompute>(plan, tmap, a, flags, stream); break;
-    case PKV_KERNEL_MMA:
-      e = plan.num_queries == 2 ? launch_one<MmaCompute2>(plan, tmap, a, flags, stream)
-                                : launch_one<MmaCompute1>(plan, tmap, a, flags, stream);
-      break;
-    default: return cudaErrorInvalidValue;
-  }
+  cudaError_t e = cudaErrorInvalidValue;
+  with_compute(plan.kernel, plan.num_queries,
+               [&](auto c) { e = launch_one<decltype(c)>(plan, tmap, a, flags, stream); });
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kKvHeads, a.batch);
@@ -1202,8 +1244,8 @@ cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
-  auto merge = a.num_queries == 2 ? (a.out_bf16 ? merge_kernel<2, true> : merge_kernel<2, false>)
-                                  : (a.out_bf16 ? merge_kernel<1, true> : merge_kernel<1, false>);
+  auto merge = a.num_queries == 1 ? (a.out_bf16 ? merge_kernel<1, true> : merge_kernel<1, false>)
+                                  : (a.out_bf16 ? merge_kernel<0, true> : merge_kernel<0, false>);
   return cudaLaunchKernelEx(&cfg, merge, a, static_cast<int32_t>(plan.grid));
 }
 

@@ -24,7 +24,7 @@ constexpr int kRowBytes = kDim * 2;               // one token of one kv head: 1
 constexpr int kTileBytes = kTokens * kRowBytes;   // (page, K|V, kv head) tile: 2 KiB
 constexpr int kRowsPerPage = 2 * kKvHeads * kTokens;  // 256 rows of 128 B
 constexpr int kPartialFloats = 2 * kGroup + kGroup * kDim;  // m[4], l[4], acc[4][64]
-constexpr int kMaxQueries = 2;   // queries per sequence in one decode launch
+constexpr int kMaxQueries = 8;   // queries per sequence in one decode launch
 
 // Sticky device error codes (first one wins).
 constexpr int32_t kErrBadPage = PKV_ERR_BAD_PAGE;

@@ -25,7 +25,7 @@ PAGE_BYTES = 32768
 
 KERNEL_AUTO, KERNEL_SIMT, KERNEL_MMA = 0, 1, 2
 DTYPE_F32, DTYPE_BF16 = 0, 1
-MAX_QUERIES = 2
+MAX_QUERIES = 8
 LAUNCH_PDL = 1
 LAUNCH_EARLY_TABLES = 2
 LAUNCH_EARLY_PAGES = 4

@@ -1,8 +1,9 @@
-"""GPU parity of the general decode call (pkv_decode): two queries per
+"""GPU parity of the general decode call (pkv_decode): several queries per
 sequence (causal among them) and BF16 output, against the FP64 oracle.
 
-Query i of two attends to the tokens t < L - 1 + i: the first query does not
-see the last token (the plainest multi-token decode).  The BF16 output must
+Query i of T attends to the tokens t < L - T + 1 + i: query T-1 sees the
+whole context, each earlier query one token fewer (the plainest multi-token
+decode, as when T drafted tokens are checked at once).  The BF16 output must
 be the FP32 result rounded to nearest even, bit for bit, so it is checked
 against the FP32 output of the same launch configuration as well as against
 the oracle (within 2e-3 plus half a BF16 step).
@@ -19,9 +20,9 @@ from tests.harness import ATOL, KERNELS, GpuCase, bits, max_err, to_dev, u16_to_
 pytestmark = pytest.mark.gpu
 
 
-def _q2(case, seed):
+def _q2(case, seed, nq=2):
     rng = np.random.default_rng(seed)
-    return bf16_bits(rng.standard_normal((len(case["seq_lens"]), 2, 32, 64)))
+    return bf16_bits(rng.standard_normal((len(case["seq_lens"]), nq, 32, 64)))
 
 
 def _run(g, q, nq, **kw):
@@ -131,5 +132,35 @@ def test_two_queries_reject_length_one_and_unsupported_forms():
                            k_new=u16_to_bf16(c["k_new"]), v_new=u16_to_bf16(c["v_new"]))
     assert e.value.status == pkv.ERR_UNSUPPORTED
     with pytest.raises(pkv.PkvError) as e:
-        _run(g, np.zeros((2, 3, 32, 64), np.uint16), 3)
+        _run(g, np.zeros((2, 9, 32, 64), np.uint16), 9)
     assert e.value.status == pkv.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("nq", [3, 4, 5, 8])
+@pytest.mark.parametrize("grid", [0, 7, 300])
+def test_up_to_eight_queries_match_oracle(nq, grid):
+    # lengths at and around page boundaries for every query: the first query's
+    # context can end one or more pages before the last one's
+    lens = [nq, 16, 16 + nq - 1, 17, 33, 0, 100, 517, 2 * 16 + nq]
+    c = make_case(lens, seed=nq * 10 + 1, spare_pages=4)
+    g = GpuCase(c)
+    q = _q2(c, nq, nq)
+    got = _f64(_run(g, q, nq, grid_ctas=grid))
+    assert pkv.get_device_error(g.pool) == 0
+    want = oracle.decode_multi(q, c["pool"], c["bt"], c["seq_lens"], 0, 0.125)
+    assert np.isfinite(got).all()
+    assert max_err(got, want) <= ATOL
+    assert not got[5].any()
+    b16 = _run(g, q, nq, grid_ctas=grid, out_dtype=torch.bfloat16)
+    assert np.array_equal(bits(b16), bf16_bits(got.astype(np.float32)))
+
+
+def test_more_queries_than_context_is_reported():
+    c = make_case([3, 40], seed=12, spare_pages=1)
+    g = GpuCase(c)
+    q = _q2(c, 6, 4)
+    got = _f64(_run(g, q, 4))
+    assert pkv.get_device_error(g.pool) == pkv.ERR_BAD_SEQ_LEN
+    assert not got[0].any()
+    want = oracle.decode_multi(q[1:], c["pool"], c["bt"][:, 1:], c["seq_lens"][1:], 0, 0.125)
+    assert max_err(got[1:], want) <= ATOL

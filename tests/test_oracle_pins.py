@@ -330,11 +330,12 @@ def _brute_multi(c, q2, scale=0.125):
     return out
 
 
-@pytest.mark.parametrize("lens", [[2], [16], [17], [18], [33, 2, 0, 40]])
-def test_decode_multi_matches_causal_bruteforce(lens):
+@pytest.mark.parametrize("lens,nq", [([2], 2), ([16], 2), ([17], 2), ([18], 2),
+                                     ([33, 2, 0, 40], 2), ([3, 17, 19], 3), ([8, 16, 23, 40], 8)])
+def test_decode_multi_matches_causal_bruteforce(lens, nq):
     c = make_case(lens, seed=sum(lens) + 3)
     rng = np.random.default_rng(len(lens))
-    q2 = bf16_bits(rng.standard_normal((len(lens), 2, H, D)))
+    q2 = bf16_bits(rng.standard_normal((len(lens), nq, H, D)))
     got = oracle.decode_multi(q2, c["pool"], c["bt"], c["seq_lens"], 0, 0.125)
     assert np.max(np.abs(got - _brute_multi(c, q2))) <= 1e-12
 
