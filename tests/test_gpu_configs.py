@@ -2,8 +2,8 @@
 oracle on the same input bits.
 
 Each test runs the workload's decode steps the way the benchmark does
-(append then decode, layer by layer, step by step) and checks, against the
-oracle:
+(append and decode, layer by layer, step by step; as two calls or as the
+fused call the benchmark times) and checks, against the oracle:
   - attention output: max abs error <= 2e-3 at the sampled (step, layer)
     points, for every sequence (or a sample of sequences for the 35 GB
     pool);
@@ -33,7 +33,7 @@ def _append_rows(host_pool, host_bt, sl_np, kb, vb, layer, rows):
     oracle.append(host_pool, host_bt[:, rows, :], sl_np[rows], kb[rows], vb[rows], layer)
 
 
-def _run(w, kernel, sample_layers, sample_steps, rows=None, flags=0, on_pool=None):
+def _run(w, kernel, sample_layers, sample_steps, rows=None, flags=0, on_pool=None, fused=False):
     """Run every step x layer of `w` on the GPU.  Returns (GPU outputs and
     oracle outputs at the sampled points for `rows`, GPU and oracle copies
     of the pages those rows use at the sampled layers)."""
@@ -53,8 +53,11 @@ def _run(w, kernel, sample_layers, sample_steps, rows=None, flags=0, on_pool=Non
         sl = to_dev(sl_np)
         for layer in range(w.num_layers):
             q, k, v = W.step_inputs(w, step, layer, dev)
-            pkv.append(pool, bt, sl, k, v, layer)
-            out = pkv.decode(q, pool, bt, sl, layer, w.scale, kernel=kernel)
+            if fused:   # the benchmark's call: append and decode in one launch
+                out = pkv.decode_append(q, k, v, pool, bt, sl, layer, w.scale, kernel=kernel)
+            else:
+                pkv.append(pool, bt, sl, k, v, layer)
+                out = pkv.decode(q, pool, bt, sl, layer, w.scale, kernel=kernel)
             if layer in sample_layers:
                 _append_rows(host_pool, host_bt, sl_np, bits(k), bits(v), layer, rows)
                 if step in sample_steps:
@@ -84,18 +87,29 @@ def test_llama1b_batch16_all_layers(kernel):
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_continuous_batching_batch64(kernel):
+@pytest.mark.parametrize("fused", [False, True])
+def test_continuous_batching_batch64(kernel, fused):
     w = W.continuous_batching()
     flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES   # as the benchmark launches it
     got, want, gp, hp, _ = _run(w, kernel, sample_layers=[0, 15],
-                                sample_steps=[1, w.num_steps], flags=flags)
+                                sample_steps=[1, w.num_steps], flags=flags, fused=fused)
     _check(got, want, gp, hp)
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_long_context_batch4(kernel):
+@pytest.mark.parametrize("fused", [False, True])
+def test_long_context_batch4(kernel, fused):
     w = W.long_context()
-    got, want, gp, hp, _ = _run(w, kernel, sample_layers=[0], sample_steps=[1])
+    flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES if fused else 0
+    got, want, gp, hp, _ = _run(w, kernel, sample_layers=[0], sample_steps=[1], flags=flags,
+                                fused=fused)
+    _check(got, want, gp, hp)
+
+
+def test_llama1b_batch16_fused_as_benchmarked():
+    w = W.llama1b()
+    got, want, gp, hp, _ = _run(w, pkv.KERNEL_AUTO, sample_layers=[0, 7, 15], sample_steps=[1],
+                                flags=pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES, fused=True)
     _check(got, want, gp, hp)
 
 
