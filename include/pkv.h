@@ -240,7 +240,11 @@ PKV_API int pkv_decode_workspace_bytes(const pkv_pool *pool, int32_t batch, size
  * weights in a fixed order (results do not depend on timing).  Device errors:
  * L < 0 or L > max_blocks*16 -> PKV_ERR_BAD_SEQ_LEN (that row is written as
  * zeros); a page outside the pool -> PKV_ERR_BAD_PAGE (that page is
- * skipped).  Requires 8 * batch * max_blocks < 2^31.
+ * skipped).  Requires 8 * batch * max_blocks < 2^31.  Every CTA keeps the
+ * batch's lengths and page-count prefix in shared memory (8 bytes per
+ * sequence): above about 4,000 sequences the tensor-core kernel runs one
+ * CTA per SM instead of two, and above about 18,000 the call returns
+ * PKV_ERR_UNSUPPORTED.
  */
 PKV_API int paged_attention_decode(const uint16_t *q, const pkv_pool *pool, const int32_t *block_tables,
                            const int32_t *seq_lens, int32_t layer, float scale, float *out,

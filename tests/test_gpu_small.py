@@ -222,3 +222,24 @@ def test_stale_workspace_contents_do_not_matter(kernel, grid, min_chunk):
     other.decode(kernel=kernel, grid_ctas=grid, min_chunk=min_chunk, workspace=ws)
     again = g.decode(scale=0.11, kernel=kernel, grid_ctas=grid, min_chunk=min_chunk, workspace=ws)
     assert np.array_equal(again, got)
+
+
+@pytest.mark.parametrize("batch", [3000, 5000])
+def test_large_batches(batch):
+    # 5,000 sequences no longer fit two tensor-core CTAs per SM (8 bytes of
+    # shared memory per sequence per CTA): the grid shrinks to one per SM
+    rng = np.random.default_rng(batch)
+    lens = [int(x) for x in rng.integers(0, 40, batch)]
+    c = make_case(lens, seed=batch, spare_pages=3)
+    g = GpuCase(c)
+    for kernel in (pkv.KERNEL_MMA, pkv.KERNEL_SIMT):
+        got = g.decode(kernel=kernel)
+        assert pkv.get_device_error(g.pool) == 0
+        assert max_err(got, g.oracle()) <= ATOL
+
+
+def test_batch_beyond_shared_memory_is_unsupported():
+    g = GpuCase(make_case([16, 16], seed=3))
+    with pytest.raises(pkv.PkvError) as e:
+        g.pool.workspace_bytes(20000)
+    assert e.value.status == pkv.ERR_UNSUPPORTED
