@@ -96,7 +96,9 @@ def measured_peaks():
 
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons, taken while the
-    timed region runs."""
+    timed region runs: sampling starts (and its first line is awaited)
+    before the region, every line is stamped with the host clock as it
+    arrives, and only lines stamped inside the region are kept."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -105,27 +107,41 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.stamped = []
+        self.lines = []
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.stamped.append((time.monotonic(), line))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+            deadline = time.monotonic() + 5.0
+            while not self.stamped and time.monotonic() < deadline:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        self.t1 = time.monotonic()
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.reader.join(timeout=5)
+        self.lines = [l for t, l in self.stamped if self.t0 <= t <= self.t1]
         return False
 
     def summary(self):
@@ -579,8 +595,12 @@ def cpu_baseline(w, pool_t, max_seconds):
 
 
 def run_reference(args, rank, world, local_rank):
-    """The oracle as the reference arm: each step is a bounded sample (one
-    whole-layer append + decode of all sequences) of the same workload."""
+    """The oracle as the reference arm: each step is a bounded sample of the
+    same workload -- append of the layer's new tokens and decode of as many
+    of its sequences (cycling through the batch) as fit the step's share of
+    --reference-seconds -- so that the whole run takes about that long
+    whatever the workload and step count."""
+    import oracle
     if rank != 0:
         return None
     w = W.make(args.workload)
@@ -588,25 +608,49 @@ def run_reference(args, rank, world, local_rank):
     if W.Workload.pool_bytes(w) > 8e9 and dev == "cpu":
         raise SystemExit("pool too large to generate on the host")
     pool_t = W.make_pool(w, dev)
-    nl = w.num_layers
+    nl, B = w.num_layers, w.batch
+    threads = os.cpu_count() or 1
+    sl = w.seq_lens(1)
+    cache = {}
+
+    def layer_inputs(l):
+        if l not in cache:
+            pool_h, bt_h = W.compact_pages(w, pool_t, range(B), [l])
+            q, k, v = W.step_inputs(w, 1, l, pool_t.device)
+            cache[l] = (pool_h, bt_h, W.bits(q), W.bits(k), W.bits(v))
+        return cache[l]
+
+    def step(l, rows):
+        pool_h0, bt_h, qb, kb, vb = layer_inputs(l)
+        pool_h = pool_h0.copy()
+        t = time.perf_counter()
+        oracle.append(pool_h, bt_h, sl, kb, vb, l)
+        oracle.decode(qb, pool_h, bt_h, sl, l, w.scale, rows=rows, nthreads=threads)
+        return time.perf_counter() - t
+
+    # calibrate: seconds per sequence of one layer
+    per_row = step(0, list(range(B))) / B
+    budget = args.reference_seconds / max(1, args.steps + args.warmup)
+    n = int(max(1, min(B, budget / max(per_row, 1e-9))))
+    rows_of = lambda i: [(i * n + j) % B for j in range(n)]
     for i in range(args.warmup):
-        oracle_sample(w, pool_t, 0.0, layers=[i % nl], max_layers=1)
+        step(i % nl, rows_of(i))
     q_tot, s_tot = 0, 0.0
-    thr = 1
     for i in range(args.steps):
-        q, s, thr, _ = oracle_sample(w, pool_t, 0.0, layers=[i % nl], max_layers=1)
-        q_tot += q
-        s_tot += s
+        s_tot += step(i % nl, rows_of(i))
+        q_tot += n
     v = q_tot / s_tot
+    sample = ("%d steps x (append of one layer's %d new tokens + decode of %d of its %d "
+              "sequences, cycling over layers and sequences)" % (args.steps, B, n, B))
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_tot / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "description": w.description, "batch": w.batch,
-                   "layers": nl, "sample": "one whole-layer append+decode per step"},
-        "cpu_baseline": {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle",
-                         "sample": "%d steps x one layer of %d sequences" % (args.steps, w.batch)},
+        "config": {"workload": w.name, "description": w.description, "batch": B,
+                   "layers": nl, "sample": sample},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -616,13 +660,15 @@ def run_reference(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="continuous_batching_b64", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "mma"])
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=60.0,
+                    help="oracle time the --impl reference run spends in its timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fill", action="store_true", help="skip the prefill fill timing")
     ap.add_argument("--early-pages", action="store_true",
