@@ -46,12 +46,17 @@
 // Two compute variants share this skeleton:
 //  - SimtCompute: CUDA-core FP32 dot products (packed FFMA2) with
 //    warp-shuffle reductions for the dot products, the max and the sum;
-//  - MmaComputeT<n>: the 16-token x 4-head tile on the tensor cores
-//    (mma.sync m16n8k16, BF16 in, FP32 accumulate) for both Q.K^T and P.V,
-//    with P split into two BF16 terms (hi + lo) so that rounding P to BF16
-//    costs no accuracy; softmax stays FP32 on the CUDA cores.  The MMA's
-//    N = 8 holds 4 heads; with n = 2 the other 4 columns carry a second query
-//    of the same sequence (causal: it sees one token more than the first).
+//  - MmaComputeT<n-tiles, one>: the 16-token x 4-head tile on the tensor
+//    cores (mma.sync m16n8k16, BF16 in, FP32 accumulate) for both Q.K^T and
+//    P.V, with P split into two BF16 terms (hi + lo) so that rounding P to
+//    BF16 costs no accuracy; softmax stays FP32 on the CUDA cores.  Each
+//    N = 8 tile holds 4 heads of two queries of the same sequence, so up to
+//    8 causal queries (each seeing one token more than the one before) share
+//    every K/V fragment; a single query leaves 4 columns zero.
+//
+// With programmatic dependent launch the kernel reads the lengths and block
+// tables, and optionally starts its first page loads, before waiting for the
+// preceding kernel of the stream (launch flags in pkv.h).
 #include <type_traits>
 
 #include "pkv_internal.cuh"
