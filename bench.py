@@ -54,14 +54,39 @@ def alg_bytes_decode(seq_lens: np.ndarray, queries: int = 1, out_bytes: int = 4)
     return int(per_seq.sum())
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without comments and with whitespace runs collapsed
+    (string and character literals kept as they are)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_digest() -> str:
-    """sha256 of the decode kernel's sources (the ncu traffic figure is only
-    valid for the sources it was captured on)."""
+    """sha256 of the decode kernel's sources without comments (the ncu
+    traffic figure is only valid for the code it was captured on)."""
     import hashlib
     h = hashlib.sha256()
     for fn in ("decode.cu", "pkv_internal.cuh"):
-        with open(os.path.join(ROOT, "paged_attention_decode_pkv_b200", "csrc", fn), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "paged_attention_decode_pkv_b200", "csrc", fn)) as f:
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()
 
 
