@@ -449,7 +449,7 @@ def run_ours(args, rank, world, local_rank):
                           (args.steps, dec_launches)),
         "clocks": clk.summary(),
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:   # the host baseline is taken at N = 1 only
         line["cpu_baseline"] = cpu_baseline(w, r.pool_t, args.cpu_seconds)
     return line
 
