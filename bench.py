@@ -11,13 +11,19 @@ fragmented block tables, 16 layers).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--kernel auto|simt|mma] [--unfused]
+                    [--queries 1..8] [--out-dtype f32|bf16] [--early-pages]
+                    [--no-pdl] [--no-fill] [--no-cpu-baseline]
 
 Prints one JSON line (rank 0).  ``value`` is decode-queries/s over all
 ranks, one query being one sequence's 32 query heads at one layer.  The
 ``roofline`` object reports the decode kernel's algorithmic HBM bytes per
 launch divided by its measured average launch time, against the measured
-HBM copy bandwidth.  ``--impl reference`` times the FP64 CPU oracle on the
-same workload instead (bounded sample per step, host cores).
+HBM copy bandwidth, with the DRAM traffic of the committed ncu capture.
+``e2e`` is the same step with its inputs and outputs crossing from and to
+pinned host memory every step; ``prefill_fill`` the page-fill bandwidth;
+``cpu_baseline`` the FP64 oracle on the host cores.  ``--impl reference``
+times the FP64 CPU oracle on the same workload instead (bounded sample per
+step, host cores).
 """
 from __future__ import annotations
 
