@@ -236,12 +236,13 @@ class Runner:
     """Device-resident state of one workload on one GPU."""
 
     def __init__(self, w: W.Workload, device, kernel: int, fused: bool, queries: int = 1,
-                 out_dtype=torch.float32):
+                 out_dtype=torch.float32, grid: int = 0):
         from paged_attention_decode_pkv_b200 import pkv
         self.pkv = pkv
         self.w = w
         self.device = device
         self.kernel = kernel
+        self.grid = grid
         self.queries = queries
         self.out_dtype = out_dtype
         # two queries per sequence: decode only (their tokens would be
@@ -267,7 +268,7 @@ class Runner:
         self.v = torch.stack([x[2] for x in ins])
         oshape = (nl, B, 32, 64) if queries == 1 else (nl, B, queries, 32, 64)
         self.out = torch.empty(oshape, dtype=out_dtype, device=device)
-        self.ws = self.pool.workspace(B, kernel, 0, queries)
+        self.ws = self.pool.workspace(B, kernel, grid, queries)
 
     def twin(self, stream):
         """A second set of step inputs and outputs (same pool, tables and
@@ -296,17 +297,19 @@ class Runner:
                 pkv.decode_general(self.q[l], self.pool, self.bt, sl, l, self.w.scale,
                                    num_queries=self.queries, out_dtype=self.out_dtype,
                                    out=self.out[l], workspace=self.ws, kernel=self.kernel,
+                                   grid_ctas=self.grid,
                                    stream=stream, **kv)
                 continue
             if self.fused:
                 pkv.decode_append(self.q[l], self.k[l], self.v[l], self.pool, self.bt, sl, l,
                                   self.w.scale, out=self.out[l], workspace=self.ws,
-                                  kernel=self.kernel, stream=stream)
+                                  kernel=self.kernel, grid_ctas=self.grid, stream=stream)
                 continue
             if not decode_only:
                 pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
             pkv.decode(self.q[l], self.pool, self.bt, sl, l, self.w.scale, out=self.out[l],
-                       workspace=self.ws, kernel=self.kernel, stream=stream)
+                       workspace=self.ws, kernel=self.kernel, grid_ctas=self.grid,
+                       stream=stream)
 
     def capture(self, stream):
         """CUDA graphs, one per lengths variant (the workload's step cycle):
@@ -346,7 +349,7 @@ def run_ours(args, rank, world, local_rank):
     w = workload_for_rank(args.workload, rank)
     fused = not args.unfused and args.queries == 1
     out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
-    r = Runner(w, device, kernel, fused, args.queries, out_dtype)
+    r = Runner(w, device, kernel, fused, args.queries, out_dtype, args.grid)
     flags = 0
     if not args.no_pdl:
         # No kernel of the step writes the lengths or the block tables.  With
@@ -707,6 +710,8 @@ def main():
     ap.add_argument("--queries", type=int, default=1, choices=range(1, 9),
                     help="queries per sequence (> 1: causal among them, decode only)")
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])
+    ap.add_argument("--grid", type=int, default=0,
+                    help="decode CTAs (0: one persistent wave over the device)")
     ap.add_argument("--unfused", action="store_true",
                     help="separate append and decode launches instead of the fused call")
     ap.add_argument("--no-pdl", action="store_true",
