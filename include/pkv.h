@@ -86,7 +86,9 @@ typedef enum {
   PKV_ERR_WORKSPACE = -6,      /* workspace missing, misaligned or too small        */
   PKV_ERR_DEVICE_TIMEOUT = -7, /* device: a bounded wait on a copy ran out           */
   PKV_ERR_BAD_SEQ_LEN = -8,    /* device: seq_len < 0 (append: < 1) or too long      */
-  PKV_ERR_TOO_LARGE = -9       /* larger than the no-alloc scratch / the whole pool */
+  PKV_ERR_TOO_LARGE = -9,      /* larger than the no-alloc scratch / the whole pool */
+  PKV_ERR_APPEND_CONFLICT = -10 /* device, with PKV_LAUNCH_CHECK_APPENDS: appends of
+                                   one call race (see pkv_pool_set_launch_flags) */
 } pkv_status;
 
 /* Launch flags for pkv_pool_set_launch_flags. */
@@ -95,6 +97,8 @@ typedef enum {
                                      tables before the preceding kernel ends */
 #define PKV_LAUNCH_EARLY_PAGES 4  /* with PDL | EARLY_TABLES: decode also starts
                                      its first page loads before then */
+#define PKV_LAUNCH_CHECK_APPENDS 8 /* check every append call for racing
+                                     appends first (debugging aid, see below) */
 #define PKV_LAUNCH_TEST_STALL (1 << 30) /* testing only: decode withholds one
                                      page so its bounded waits run out (~1 s)
                                      and it reports PKV_ERR_DEVICE_TIMEOUT */
@@ -149,6 +153,17 @@ PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
  * the pool pages it reads: true when that kernel is the previous layer's
  * decode or merge, or a projection that writes q; false when it is a
  * pkv_append or pkv_fill into this layer (use the fused call instead).
+ * PKV_LAUNCH_CHECK_APPENDS makes pkv_append and the fused calls
+ * (paged_attention_decode_append[_ex], pkv_decode with k_new) first launch a
+ * check, on the same stream, that records PKV_ERR_APPEND_CONFLICT when the
+ * call's result would be undefined: two sequences append to the same slot,
+ * or (fused calls only) a sequence appends to a slot that lies inside a
+ * context the call reads -- another sequence's, or its own through a page
+ * its table names twice.  A shared page whose slots are only read (a common
+ * prefix) is fine.  Sequences whose own append is invalid are left to the
+ * append's own errors.  The check only reports: the append still runs.  It
+ * costs batch x (batch, or table entries when fused) comparisons, so it is
+ * meant for debugging, not for the hot path.
  * PKV_LAUNCH_TEST_STALL exists only to test the device-timeout path: the
  * decode kernel never fills one shared-memory stage, every wait on it gives
  * up after about a second, the kernel exits early with garbage output and
@@ -156,7 +171,8 @@ PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
  * usable.
  * flags: 0, PKV_LAUNCH_PDL, PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES or
  * PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES | PKV_LAUNCH_EARLY_PAGES,
- * optionally | PKV_LAUNCH_TEST_STALL, else PKV_ERR_INVALID_ARG.
+ * each optionally | PKV_LAUNCH_CHECK_APPENDS and | PKV_LAUNCH_TEST_STALL,
+ * else PKV_ERR_INVALID_ARG.
  */
 PKV_API int pkv_pool_set_launch_flags(pkv_pool *pool, int32_t flags);
 
@@ -165,7 +181,8 @@ PKV_API int pkv_pool_set_launch_flags(pkv_pool *pool, int32_t flags);
  * L = seq_lens[b], copy k_new[b][g][:] and v_new[b][g][:] for all 8 kv
  * heads into slot (L-1) % 16 of page block_tables[layer][b][(L-1)/16].
  * Bit copies.  seq_lens is not modified (the caller advances it).  Two
- * sequences appending into the same page slot is undefined.  Device errors:
+ * sequences appending into the same page slot is undefined (detected with
+ * PKV_LAUNCH_CHECK_APPENDS).  Device errors:
  * L < 1 or L > max_blocks*16 -> PKV_ERR_BAD_SEQ_LEN, page outside the pool
  * -> PKV_ERR_BAD_PAGE; that sequence is skipped.
  */
@@ -279,7 +296,8 @@ PKV_API int paged_attention_decode_ex(const uint16_t *q, const pkv_pool *pool,
  * Differences from the two calls: a sequence with L = 0 gets no append and
  * a zero output row without an error (an idle batch slot); the appended
  * slot must not lie in another sequence's context in this call (a page that
- * several sequences read is read-only).  Errors and outputs otherwise as
+ * several sequences read is read-only; detected with
+ * PKV_LAUNCH_CHECK_APPENDS).  Errors and outputs otherwise as
  * pkv_append and paged_attention_decode; a page outside the pool is neither
  * read nor written.  Workspace: pkv_decode_workspace_bytes[_ex].
  */

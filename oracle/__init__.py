@@ -4,4 +4,5 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg may import this package.  The product path (the CUDA library and its
 binding) never does.
 """
-from .oracle import append, fill, gather, decode, decode_multi, OracleError  # noqa: F401
+from .oracle import (append, append_conflict, fill, gather, decode, decode_multi,  # noqa: F401
+                     OracleError)

@@ -4,7 +4,8 @@ Arrays are numpy: the pool is uint16 [num_pages, 2, 8, 16, 64] (BF16 bits,
 layout page[kv][kv_head][slot][d]); block tables int32
 [num_layers, batch, max_blocks]; seq_lens int32 [batch] (length after the
 step's append); q uint16 [batch, 32, 64]; k_new / v_new uint16 [batch, 8, 64].
-Outputs of decode are float64 [batch, 32, 64].
+Outputs of decode are float64 [batch, 32, 64].  append_conflict (which
+appends of one call race) is plain Python on the same arrays.
 """
 import ctypes
 import os
@@ -150,3 +151,47 @@ def decode_multi(q, pool, block_tables, seq_lens, layer, scale, nthreads=None):
         out[:, i] = decode(np.ascontiguousarray(q[:, i]), pool, block_tables, li, layer, scale,
                            nthreads=nthreads)
     return out
+
+
+def append_conflict(block_tables, seq_lens, layer, num_pages, fused):
+    """True when the appends of one call race, by the definition of an append.
+
+    Sequence b with 1 <= L_b <= 16 * max_blocks writes position L_b - 1: slot
+    (L_b - 1) % 16 of page block_tables[layer][b][(L_b - 1) // 16] ("Curso
+    gratuito recorre la inferencia de LLM...", section on the KV cache), when
+    that page lies in the pool; other sequences write nothing.
+      plain append (fused=False): two sequences write the same (page, slot).
+      fused append + decode (fused=True): some written (page, slot) is read by
+        the call, other than by its writer at its own new position: sequence
+        c (1 <= L_c <= 16 * max_blocks) reads slot t % 16 of page
+        block_tables[layer][c][t // 16] for every t < L_c.  Two writes to one
+        slot are the case where one writer reads the other's new position.
+    Plain Python over the (page -> writes) map; fine up to full workload sizes.
+    """
+    bt = np.asarray(block_tables)[layer]
+    lens = np.asarray(seq_lens)
+    batch, max_blocks = bt.shape
+    writes = {}   # page -> [(slot, writer)]
+    for b in range(batch):
+        L = int(lens[b])
+        if not 1 <= L <= 16 * max_blocks:
+            continue
+        page = int(bt[b, (L - 1) // 16])
+        if 0 <= page < num_pages:
+            writes.setdefault(page, []).append(((L - 1) % 16, b))
+    if not fused:
+        for lst in writes.values():
+            slots = [s for s, _ in lst]
+            if len(set(slots)) != len(slots):
+                return True
+        return False
+    for c in range(batch):
+        L = int(lens[c])
+        if not 1 <= L <= 16 * max_blocks:
+            continue
+        for j in range((L + 15) // 16):
+            for s, b in writes.get(int(bt[c, j]), ()):
+                t = 16 * j + s
+                if t < L and not (b == c and t == L - 1):
+                    return True
+    return False

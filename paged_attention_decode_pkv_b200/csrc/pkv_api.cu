@@ -6,6 +6,7 @@
 #include <mutex>
 #include <new>
 
+#include "append_check.cuh"
 #include "pkv_internal.cuh"
 
 struct pkv_pool {
@@ -177,6 +178,13 @@ int pkv_append(pkv_pool* pool, const int32_t* block_tables, const int32_t* seq_l
   if (s != PKV_OK) return s;
   if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return PKV_ERR_INVALID_ARG;
   if (batch > 2147483647 / 2) return PKV_ERR_UNSUPPORTED;
+  if (pool->launch_flags & PKV_LAUNCH_CHECK_APPENDS) {
+    s = from_cuda(pkv::launch_append_check(layer_slab(block_tables, layer, batch, max_blocks),
+                                           seq_lens, pool->d_err, batch, max_blocks,
+                                           pool->num_pages, false,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+    if (s != PKV_OK) return s;
+  }
   return from_cuda(pkv::launch_append(
       reinterpret_cast<const __nv_bfloat16*>(k_new), reinterpret_cast<const __nv_bfloat16*>(v_new),
       static_cast<__nv_bfloat16*>(pool->data), layer_slab(block_tables, layer, batch, max_blocks),
@@ -205,7 +213,7 @@ int pkv_fill(pkv_pool* pool, const int32_t* block_tables, const int32_t* cu_toke
 
 int pkv_pool_set_launch_flags(pkv_pool* pool, int32_t flags) {
   if (!pool || (flags & ~(PKV_LAUNCH_PDL | PKV_LAUNCH_EARLY_TABLES | PKV_LAUNCH_EARLY_PAGES |
-                          PKV_LAUNCH_TEST_STALL)))
+                          PKV_LAUNCH_CHECK_APPENDS | PKV_LAUNCH_TEST_STALL)))
     return PKV_ERR_INVALID_ARG;
   if ((flags & PKV_LAUNCH_EARLY_TABLES) && !(flags & PKV_LAUNCH_PDL)) return PKV_ERR_INVALID_ARG;
   if ((flags & PKV_LAUNCH_EARLY_PAGES) && !(flags & PKV_LAUNCH_EARLY_TABLES))
@@ -271,6 +279,12 @@ int decode_common(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_ne
   a.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
   a.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
   a.pool = static_cast<__nv_bfloat16*>(pool->data);
+  if (k_new && (pool->launch_flags & PKV_LAUNCH_CHECK_APPENDS)) {
+    s = from_cuda(pkv::launch_append_check(a.bt, seq_lens, pool->d_err, batch, max_blocks,
+                                           pool->num_pages, true,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+    if (s != PKV_OK) return s;
+  }
   return from_cuda(pkv::launch_decode(plan, pool->tmap, a, pool->launch_flags,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -453,6 +467,7 @@ const char* pkv_status_string(int status) {
     case PKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case PKV_ERR_BAD_SEQ_LEN: return "sequence length out of range";
     case PKV_ERR_TOO_LARGE: return "request larger than the fixed no-alloc scratch or the whole pool";
+    case PKV_ERR_APPEND_CONFLICT: return "appends of one call race (same slot, or a slot another context reads)";
     default: return "unknown status";
   }
 }

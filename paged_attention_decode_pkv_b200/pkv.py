@@ -29,6 +29,7 @@ MAX_QUERIES = 8
 LAUNCH_PDL = 1
 LAUNCH_EARLY_TABLES = 2
 LAUNCH_EARLY_PAGES = 4
+LAUNCH_CHECK_APPENDS = 8
 LAUNCH_TEST_STALL = 1 << 30
 
 OK = 0
@@ -41,6 +42,7 @@ ERR_WORKSPACE = -6
 ERR_DEVICE_TIMEOUT = -7
 ERR_BAD_SEQ_LEN = -8
 ERR_TOO_LARGE = -9
+ERR_APPEND_CONFLICT = -10
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTS = (

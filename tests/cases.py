@@ -67,3 +67,31 @@ def contiguous_kv(case, layer=0):
         V = case["pool"][pages, 1, :, t % T, :]
         out.append((bf16_to_f64(K).transpose(1, 0, 2), bf16_to_f64(V).transpose(1, 0, 2)))
     return out
+
+
+# Hand-worked append-race cases: (name, block-table rows [batch][max_blocks],
+# lengths after the append, race under pkv_append, race under the fused
+# call), over a pool of APPEND_CASE_PAGES pages.  Sequence b writes slot
+# (L-1) % 16 of page row[(L-1) // 16]; the fused call also reads slots
+# t % 16 of pages row[t // 16] for t < L.
+APPEND_CASE_PAGES = 8
+APPEND_CONFLICT_CASES = [
+    # (0,4) and (3,3): distinct pages, each read only by its writer
+    ("distinct pages", [[0, 1], [2, 3]], [5, 20], False, False),
+    # both write (5,2)
+    ("same slot", [[5, 0], [5, 1]], [3, 3], True, True),
+    # writes (5,3) and (5,5); sequence 1 reads slots 0..5 of page 5
+    ("same page, other slots", [[5, 0], [5, 1]], [4, 6], False, True),
+    # page 7 is a prefix both read in full; the writes go to pages 1 and 2
+    ("shared read-only prefix", [[7, 1], [7, 2]], [20, 18], False, False),
+    # sequence 1 (L = 0) names page 4 but reads and writes nothing
+    ("idle slot names the page", [[4, 0], [4, 0]], [11, 0], False, False),
+    # page 3 named twice: the write (3,3) at t = 19 lands on t = 3 of the same context
+    ("page named twice by one table", [[3, 3], [0, 1]], [20, 2], False, True),
+    # sequence 1's page is outside the pool: no write; sequence 2 writes (2,0)
+    ("invalid page is no write", [[6, 0], [99, 0], [2, 0]], [9, 1, 1], False, False),
+    # both name page 99, outside the pool: neither writes
+    ("two writes outside the pool", [[99, 0], [99, 0]], [1, 1], False, False),
+    # three writers, two of them on (1,15); the third on (1,0) is read by both
+    ("three writers", [[1, 0], [0, 1], [2, 1]], [16, 32, 17], True, True),
+]

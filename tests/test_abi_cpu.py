@@ -39,6 +39,19 @@ def test_status_strings():
     assert pkv.status_string(0) == "ok"
     assert "outside the pool" in pkv.status_string(pkv.ERR_BAD_PAGE)
     assert pkv.status_string(12345) == "unknown status"
+    assert "race" in pkv.status_string(pkv.ERR_APPEND_CONFLICT)
+
+
+def test_binding_constants_match_the_header():
+    """Every PKV_ERR_* code and PKV_LAUNCH_* flag of the header has the same
+    value under the same name in the Python binding."""
+    from paged_attention_decode_pkv_b200 import pkv
+    src = open(os.path.join(ROOT, "include", "pkv.h")).read()
+    errs = dict(re.findall(r"\bPKV_(ERR_\w+)\s*=\s*(-?\d+)", src))
+    flags = dict(re.findall(r"#define\s+PKV_(LAUNCH_\w+)\s+(\(?[\d\s<]+\)?)", src))
+    assert len(errs) >= 10 and len(flags) >= 5
+    for name, value in list(errs.items()) + list(flags.items()):
+        assert getattr(pkv, name) == eval(value), name
 
 
 def test_pool_create_rejects_bad_shapes_and_null_out():
