@@ -86,8 +86,8 @@ def test_random_tables_match_oracle(fused):
         lens = rng.integers(0, 16 * mb + 1, size=batch).astype(np.int32)
         if rng.random() < 0.5:
             lens = np.minimum(lens, rng.integers(0, 20, size=batch)).astype(np.int32)
-        if not fused:
-            lens = np.maximum(lens, 1).astype(np.int32)
+        if not fused:   # plain appends race only on a shared slot: favour short contexts
+            lens = np.maximum(lens if rng.random() < 0.3 else lens % 3, 1).astype(np.int32)
         want = _allowed(bt, lens, pages, fused)
         got = _status(bt, lens, pages, fused, seed=i)
         assert got in want, (i, bt, lens, pages, got, want)
