@@ -182,7 +182,7 @@ def test_programmatic_dependent_launch_keeps_results(kernel):
     with pytest.raises(pkv.PkvError):
         g.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_PAGES)   # needs early tables
     with pytest.raises(pkv.PkvError):
-        g.pool.set_launch_flags(8)
+        g.pool.set_launch_flags(16)   # no such flag
     g.pool.set_launch_flags(pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES)
     for _ in range(3):
         pkv.append(g.pool, g.bt, g.sl, u16_to_bf16(c["k_new"]), u16_to_bf16(c["v_new"]), 0)
