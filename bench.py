@@ -12,10 +12,14 @@ fragmented block tables, 16 layers).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--kernel auto|simt|mma] [--unfused]
                     [--queries 1..8] [--out-dtype f32|bf16] [--early-pages]
-                    [--no-pdl] [--no-fill] [--no-cpu-baseline]
+                    [--grid CTAS] [--no-pdl] [--no-fill] [--no-cpu-baseline]
+                    [--e2e-steps N] [--cpu-seconds S] [--reference-seconds S]
 
 Prints one JSON line (rank 0).  ``value`` is decode-queries/s over all
-ranks, one query being one sequence's 32 query heads at one layer.  The
+ranks, one query being one sequence's 32 query heads at one layer
+(``head_queries_per_s`` counts heads, ``tokens_per_s`` sequences' tokens
+per whole-model step; ``append``, in --unfused runs, the separate append's
+share of a layer).  The
 ``roofline`` object reports the decode kernel's algorithmic HBM bytes per
 launch divided by its measured average launch time, against the measured
 HBM copy bandwidth, with the DRAM traffic of the committed ncu capture.
@@ -446,6 +450,8 @@ def run_ours(args, rank, world, local_rank):
             "launches": dec_launches,
         },
         "decode_queries_per_s": w.batch * r.queries / avg_dec_s,
+        "head_queries_per_s": value * 32,
+        "tokens_per_s": value / w.num_layers,
         "e2e": e2e,
         "prefill_fill": fill,
         "gpu_launches": (args.steps * w.num_layers * (2 if fused or r.queries > 1 else 3) +
@@ -458,6 +464,14 @@ def run_ours(args, rank, world, local_rank):
                           (args.steps, dec_launches)),
         "clocks": clk.summary(),
     }
+    if not fused and r.queries == 1:
+        # the separate append's share of a layer: full step replays minus the
+        # replays of the same decode + merge launches alone
+        line["append"] = {
+            "kernel": "append_kernel", "us_per_launch":
+                (t0.elapsed_time(t1) - d0.elapsed_time(d1)) / dec_launches * 1e3,
+            "bytes_per_launch": w.batch * (2 * 2048 + 8),
+            "how": "unfused step time minus decode + merge time, per layer (PDL-chained)"}
     if not args.no_cpu_baseline and world == 1:   # the host baseline is taken at N = 1 only
         line["cpu_baseline"] = cpu_baseline(w, r.pool_t, args.cpu_seconds)
     return line
@@ -589,7 +603,8 @@ def run_fill(r: Runner, stream, steps, device):
 
 # ------------------------------------------------------------ oracle arms --
 
-def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None, max_layers=None):
+def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None, max_layers=None,
+                  threads=None):
     """Time the FP64 oracle on whole-layer append + decode of step 1 (all
     sequences of the batch), cycling over `layers`, until `max_seconds` of
     oracle time have passed (at least one layer; at most `max_layers`).
@@ -598,7 +613,7 @@ def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None, max_la
     threads, layer-decodes done)."""
     import oracle
     layers = list(range(w.num_layers)) if layers is None else list(layers)
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     sl = w.seq_lens(1)
     cache = {}
     done, secs = 0, 0.0
@@ -621,10 +636,14 @@ def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None, max_la
 
 def cpu_baseline(w, pool_t, max_seconds):
     q, s, thr, layers = oracle_sample(w, pool_t, max_seconds, max_layers=4096)
+    q1, s1, _, layers1 = oracle_sample(w, pool_t, max_seconds / 4, max_layers=4096, threads=1)
     return {"value": q / s, "unit": UNIT, "cores": thr, "kind": "oracle",
             "sample": "%d whole-layer append+decode(s) of step 1, cycling over the %d layers "
                       "(%d sequences each), %.1f s of FP64 oracle work" %
-                      (layers, w.num_layers, w.batch, s)}
+                      (layers, w.num_layers, w.batch, s),
+            "single_core_value": q1 / s1,
+            "single_core_sample": "%d whole-layer append+decode(s) on 1 thread, %.1f s" %
+                                  (layers1, s1)}
 
 
 def run_reference(args, rank, world, local_rank):
