@@ -59,21 +59,29 @@ __global__ void __launch_bounds__(128) append_kernel(const uint4* __restrict__ k
 
 // Fill: one CTA per kFillRowsPerCta consecutive source rows t (rows
 // [0, total) of k_src / v_src).  512 threads = 4 row lanes x (K|V) x 8 kv
-// heads x 8 chunks of 16 B; each lane moves kFillRowsPerLane rows, with all
-// its loads issued first.  While they are in flight, one thread per row maps
-// the row to its destination -- row t belongs to the last sequence b with
-// cu[b] <= t (binary search over cu), goes to position start[b] + t - cu[b],
-// so to slot pos % 16 of page bt[b][pos / 16] -- and shares it through
-// shared memory: the index loads are issued once per row, not once per
-// 16-byte chunk.  The grid follows the row count, not (sequence x longest
-// prompt), so a batch of mixed prompt lengths launches no empty CTAs.
+// heads x 8 chunks of 16 B; each lane moves kFillRowsPerLane rows, and all
+// their loads go out first: they depend on nothing but the row count.
+// While they are in flight, one thread per row maps the row to its
+// destination -- row t belongs to the last sequence b with cu[b] <= t,
+// goes to position start[b] + t - cu[b], so to slot pos % 16 of page
+// bt[b][pos / 16] -- and shares it through shared memory, so the index
+// loads are issued once per row, not once per 16-byte chunk.  For batches
+// of fewer than 512 sequences the CTA first copies cu and start into
+// shared memory (one round of loads, beside the data loads) and searches
+// there, so a row's destination costs two dependent rounds of memory
+// latency (cu and start, then the block-table entry) instead of one per
+// step of a binary search in global memory.  The grid follows the row
+// count, not (sequence x longest prompt), so a batch of mixed prompt
+// lengths launches no empty CTAs.
 constexpr int kFillThreads = 512;
 constexpr int kFillLanes = kFillThreads / 128;
 constexpr int kFillRowsPerLane = 4;
 constexpr int kFillRowsPerCta = kFillLanes * kFillRowsPerLane;
+constexpr int kFillSmemBatch = kFillThreads - 1;   // largest batch searched in shared memory
 
-__device__ __forceinline__ int32_t fill_seq_of(const int32_t* __restrict__ cu, int32_t batch,
-                                               int32_t t) {
+// The last b in [0, batch) with cu[b] <= t, for cu non-decreasing (global
+// or shared memory).
+__device__ __forceinline__ int32_t fill_seq_of(const int32_t* cu, int32_t batch, int32_t t) {
   int32_t lo = 0, hi = batch;   // cu[lo] <= t < cu[hi] when cu is non-decreasing
   while (hi - lo > 1) {
     const int32_t mid = (lo + hi) >> 1;
@@ -89,20 +97,14 @@ __global__ void __launch_bounds__(kFillThreads)
                 int32_t* __restrict__ err, int32_t batch, int32_t max_blocks,
                 int32_t num_pages, int32_t total) {
   __shared__ int64_t s_row[kFillRowsPerCta];   // pool row of (page, K, head 0, slot), or -1
+  __shared__ int32_t s_cu[kFillSmemBatch + 1];
+  __shared__ int32_t s_start[kFillSmemBatch];
   pdl_wait();
   pdl_trigger();
   const int tid = threadIdx.x;
   const int kv = (tid >> 6) & 1;
   const int g = (tid >> 3) & 7;
   const int c = tid & 7;
-  // the rows the caller passed must be exactly the rows cu describes
-  if (cu[0] != 0 || cu[batch] != total) {   // uniform over the grid
-    if (blockIdx.x == 0 && tid == 0) record_error(err, kErrBadLen);
-    return;
-  }
-  // a decreasing cu makes the row -> sequence map ambiguous: report it
-  for (int32_t b = blockIdx.x * blockDim.x + tid; b < batch; b += gridDim.x * blockDim.x)
-    if (cu[b + 1] < cu[b]) record_error(err, kErrBadLen);
   const int32_t row0 = blockIdx.x * kFillRowsPerCta;
   const uint4* src = kv ? v_src : k_src;
   uint4 val[kFillRowsPerLane];
@@ -111,12 +113,29 @@ __global__ void __launch_bounds__(kFillThreads)
     const int32_t t = row0 + (tid >> 7) + kFillLanes * j;
     if (t < total) val[j] = __ldcs(src + (static_cast<int64_t>(t) * kKvHeads + g) * 8 + c);
   }
+  const bool staged = batch <= kFillSmemBatch;   // uniform over the grid
+  if (staged) {
+    for (int i = tid; i <= batch; i += kFillThreads) {
+      s_cu[i] = cu[i];
+      if (i < batch) s_start[i] = start[i];
+    }
+  }
+  // a decreasing cu makes the row -> sequence map ambiguous: report it
+  for (int32_t b = blockIdx.x * blockDim.x + tid; b < batch; b += gridDim.x * blockDim.x)
+    if (cu[b + 1] < cu[b]) record_error(err, kErrBadLen);
+  __syncthreads();
+  const int32_t* cu_s = staged ? s_cu : cu;
+  // the rows the caller passed must be exactly the rows cu describes
+  if (cu_s[0] != 0 || cu_s[batch] != total) {   // uniform over the grid: nothing is written
+    if (blockIdx.x == 0 && tid == 0) record_error(err, kErrBadLen);
+    return;
+  }
   if (tid < kFillRowsPerCta) {
     const int32_t t = row0 + tid;
     int64_t row = -1;
     if (t < total) {
-      const int32_t b = fill_seq_of(cu, batch, t);
-      const int32_t c0 = cu[b], c1 = cu[b + 1], s0 = start[b];
+      const int32_t b = fill_seq_of(cu_s, batch, t);
+      const int32_t c0 = cu_s[b], c1 = cu_s[b + 1], s0 = staged ? s_start[b] : start[b];
       if (t < c0 || t >= c1 || s0 < 0 ||
           static_cast<int64_t>(s0) + (c1 - c0) > static_cast<int64_t>(max_blocks) * kTokens) {
         record_error(err, kErrBadLen);

@@ -54,6 +54,23 @@ def test_fill_bit_exact_whole_pool(counts, starts):
     assert np.array_equal(bits(g.pool_t).reshape(host.shape), host)
 
 
+@pytest.mark.parametrize("batch", [510, 511, 512, 1300])
+def test_fill_batches_around_the_shared_memory_index(batch):
+    """Up to 511 sequences the CTA searches cu in shared memory, from 512 on
+    in global memory: both bit-exact, with empty, short and page-crossing
+    prompts and starts inside a page."""
+    rng = np.random.default_rng(batch)
+    counts = [int(x) for x in rng.choice([0, 1, 3, 16, 17, 40], batch)]
+    starts = [int(x) for x in rng.integers(0, 20, batch)]
+    c = make_case([s + n for s, n in zip(starts, counts)], seed=batch, spare_pages=2)
+    g = GpuCase(c)
+    host = c["pool"].copy()
+    _fill_both(g, host, counts, starts, 0, rng)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error(g.pool) == 0
+    assert np.array_equal(bits(g.pool_t).reshape(host.shape), host)
+
+
 def test_long_ragged_fill_spans_many_ctas():
     # ~8600 rows = 536 CTAs of 16 rows and a ragged last CTA; prompts cross
     # many page boundaries, and start mid page
