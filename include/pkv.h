@@ -153,17 +153,22 @@ PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
  * the pool pages it reads: true when that kernel is the previous layer's
  * decode or merge, or a projection that writes q; false when it is a
  * pkv_append or pkv_fill into this layer (use the fused call instead).
- * PKV_LAUNCH_CHECK_APPENDS makes pkv_append and the fused calls
+ * PKV_LAUNCH_CHECK_APPENDS makes pkv_append, pkv_fill and the fused calls
  * (paged_attention_decode_append[_ex], pkv_decode with k_new) first launch a
  * check, on the same stream, that records PKV_ERR_APPEND_CONFLICT when the
  * call's result would be undefined: two sequences append to the same slot,
  * or (fused calls only) a sequence appends to a slot that lies inside a
  * context the call reads -- another sequence's, or its own through a page
- * its table names twice.  A shared page whose slots are only read (a common
- * prefix) is fine.  Sequences whose own append is invalid are left to the
- * append's own errors.  The check only reports: the append still runs.  It
- * costs batch x (batch, or table entries when fused) comparisons, so it is
- * meant for debugging, not for the hot path.
+ * its table names twice; for pkv_fill, two tokens (of two sequences, or of
+ * one whose table names a page twice) are written to the same slot.  A
+ * shared page whose slots are only read (a common prefix) is fine.
+ * Sequences and tokens that the call itself skips as invalid are left to
+ * its own errors.  The check only reports: the write still runs.  It costs
+ * batch x (batch, or table entries when fused) comparisons, and for
+ * pkv_fill a clear of a slot bitmap (2 bytes per page) plus one atomic per
+ * token, so it is meant for debugging, not for the hot path.  Setting the
+ * flag allocates that bitmap once (freed with the pool): the only device
+ * allocation outside pool creation; PKV_ERR_CUDA if it fails.
  * PKV_LAUNCH_TEST_STALL exists only to test the device-timeout path: the
  * decode kernel never fills one shared-memory stage, every wait on it gives
  * up after about a second, the kernel exits early with garbage output and
@@ -209,7 +214,7 @@ PKV_API int pkv_append(pkv_pool *pool, const int32_t *block_tables, const int32_
  * PKV_ERR_BAD_PAGE (that token is skipped).  Whatever the device inputs, no
  * source row outside [0, total_tokens) is read and nothing outside the pool
  * is written.  The positions of different sequences must name different
- * slots.  Stream ordered; PDL-chained like pkv_append when the pool's PDL
+ * slots (detected with PKV_LAUNCH_CHECK_APPENDS).  Stream ordered; PDL-chained like pkv_append when the pool's PDL
  * flag is set.  max_blocks * 16 must fit in int32.
  */
 PKV_API int pkv_fill(pkv_pool *pool, const int32_t *block_tables, const int32_t *cu_tokens,

@@ -4,8 +4,9 @@ Arrays are numpy: the pool is uint16 [num_pages, 2, 8, 16, 64] (BF16 bits,
 layout page[kv][kv_head][slot][d]); block tables int32
 [num_layers, batch, max_blocks]; seq_lens int32 [batch] (length after the
 step's append); q uint16 [batch, 32, 64]; k_new / v_new uint16 [batch, 8, 64].
-Outputs of decode are float64 [batch, 32, 64].  append_conflict (which
-appends of one call race) is plain Python on the same arrays.
+Outputs of decode are float64 [batch, 32, 64].  append_conflict and
+fill_conflict (which writes of one call race) are plain Python on the same
+arrays.
 """
 import ctypes
 import os
@@ -194,4 +195,40 @@ def append_conflict(block_tables, seq_lens, layer, num_pages, fused):
                 t = 16 * j + s
                 if t < L and not (b == c and t == L - 1):
                     return True
+    return False
+
+
+def fill_conflict(block_tables, cu, start, layer, num_pages):
+    """True when two tokens of one fill call are written to the same slot.
+
+    Token i of sequence b (i < cu[b+1] - cu[b]) goes to position start[b] + i,
+    slot (start[b] + i) % 16 of page block_tables[layer][b][(start[b] + i) // 16]
+    ("Curso gratuito recorre la inferencia de LLM...", section on the KV
+    cache).  A sequence with start[b] < 0 or an end beyond 16 * max_blocks
+    writes nothing, nor does a token whose page lies outside the pool; when
+    cu does not start at 0 the call writes nothing at all.  cu must be
+    non-decreasing (ValueError otherwise: which tokens are written is then
+    unspecified).
+    """
+    bt = np.asarray(block_tables)[layer]
+    cu = np.asarray(cu)
+    st = np.asarray(start)
+    batch, max_blocks = bt.shape
+    if np.any(np.diff(cu) < 0):
+        raise ValueError("cu_tokens decreases")
+    if cu[0] != 0:
+        return False
+    seen = set()
+    for b in range(batch):
+        n = int(cu[b + 1] - cu[b])
+        s0 = int(st[b])
+        if s0 < 0 or s0 + n > 16 * max_blocks:
+            continue
+        for pos in range(s0, s0 + n):
+            page = int(bt[b, pos // 16])
+            if not 0 <= page < num_pages:
+                continue
+            if (page, pos % 16) in seen:
+                return True
+            seen.add((page, pos % 16))
     return False

@@ -22,7 +22,12 @@
 // Sequences whose own append is invalid (length or page out of range) are
 // skipped; the append itself reports them.  The cost is entries x batch
 // comparisons: a debugging aid, not a hot-path step.
+//
+// pkv_fill writes many tokens per sequence, so its check marks the written
+// slots in a bitmap of the pool (one bit per slot, two bytes per page)
+// instead of comparing pairs.
 #include "append_check.cuh"
+#include "fill_map.cuh"
 #include "pkv_internal.cuh"
 
 namespace pkv {
@@ -94,7 +99,54 @@ __global__ void __launch_bounds__(kCheckThreads)
   if (conflict) record_error(err, kErrAppendConflict);
 }
 
+// Fill: every valid source row t marks bit (page * 16 + slot) of `bits`
+// (zeroed before the launch); a bit that was already set means two rows --
+// of two sequences, or of one whose table names a page twice -- write one
+// slot.  Rows are mapped exactly as pkv_fill maps them, and rows that
+// pkv_fill skips (bad range, page outside the pool) mark nothing.
+__global__ void __launch_bounds__(kCheckThreads)
+    fill_check_kernel(const int32_t* __restrict__ bt, const int32_t* __restrict__ cu,
+                      const int32_t* __restrict__ start, uint32_t* __restrict__ bits,
+                      int32_t* __restrict__ err, int32_t batch, int32_t max_blocks,
+                      int32_t num_pages, int32_t total) {
+  if (cu[0] != 0 || cu[batch] != total) return;   // pkv_fill writes nothing
+  bool conflict = false;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int32_t t = static_cast<int32_t>(e);
+    const int32_t b = fill_seq_of(cu, batch, t);
+    const int32_t c0 = cu[b], c1 = cu[b + 1], s0 = start[b];
+    if (t < c0 || t >= c1 || s0 < 0 ||
+        static_cast<int64_t>(s0) + (c1 - c0) > static_cast<int64_t>(max_blocks) * kTokens)
+      continue;
+    const int32_t pos = s0 + (t - c0);
+    const int32_t page = bt[static_cast<int64_t>(b) * max_blocks + pos / kTokens];
+    if (page < 0 || page >= num_pages) continue;
+    const int64_t idx = static_cast<int64_t>(page) * kTokens + pos % kTokens;
+    const uint32_t bit = 1u << (idx & 31);
+    if (atomicOr(bits + (idx >> 5), bit) & bit) conflict = true;
+  }
+  if (conflict) record_error(err, kErrAppendConflict);
+}
+
 }  // namespace
+
+size_t fill_check_bitmap_bytes(int32_t num_pages) {
+  return (static_cast<size_t>(num_pages) * kTokens + 31) / 32 * sizeof(uint32_t);
+}
+
+cudaError_t launch_fill_check(const int32_t* bt, const int32_t* cu, const int32_t* start,
+                              uint32_t* bits, int32_t* err, int32_t batch, int32_t max_blocks,
+                              int32_t num_pages, int32_t total_tokens, cudaStream_t stream) {
+  if (batch == 0 || total_tokens == 0) return cudaSuccess;
+  cudaError_t e = cudaMemsetAsync(bits, 0, fill_check_bitmap_bytes(num_pages), stream);
+  if (e != cudaSuccess) return e;
+  const int64_t want = (static_cast<int64_t>(total_tokens) + kCheckThreads - 1) / kCheckThreads;
+  const int grid = static_cast<int>(want < kCheckMaxCtas ? want : kCheckMaxCtas);
+  fill_check_kernel<<<grid, kCheckThreads, 0, stream>>>(bt, cu, start, bits, err, batch,
+                                                        max_blocks, num_pages, total_tokens);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_append_check(const int32_t* bt, const int32_t* seq_lens, int32_t* err,
                                 int32_t batch, int32_t max_blocks, int32_t num_pages,

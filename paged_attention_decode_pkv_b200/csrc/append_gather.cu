@@ -18,6 +18,7 @@
 // All three are pure 16-byte copies: 8 consecutive threads move one 128-byte row
 // (one token of one kv head), so every warp access is four full 128-byte
 // lines.
+#include "fill_map.cuh"
 #include "pkv_internal.cuh"
 
 namespace pkv {
@@ -78,17 +79,6 @@ constexpr int kFillLanes = kFillThreads / 128;
 constexpr int kFillRowsPerLane = 4;
 constexpr int kFillRowsPerCta = kFillLanes * kFillRowsPerLane;
 constexpr int kFillSmemBatch = kFillThreads - 1;   // largest batch searched in shared memory
-
-// The last b in [0, batch) with cu[b] <= t, for cu non-decreasing (global
-// or shared memory).
-__device__ __forceinline__ int32_t fill_seq_of(const int32_t* cu, int32_t batch, int32_t t) {
-  int32_t lo = 0, hi = batch;   // cu[lo] <= t < cu[hi] when cu is non-decreasing
-  while (hi - lo > 1) {
-    const int32_t mid = (lo + hi) >> 1;
-    if (cu[mid] <= t) lo = mid; else hi = mid;
-  }
-  return lo;
-}
 
 __global__ void __launch_bounds__(kFillThreads)
     fill_kernel(const uint4* __restrict__ k_src, const uint4* __restrict__ v_src,

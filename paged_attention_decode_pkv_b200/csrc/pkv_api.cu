@@ -17,6 +17,7 @@ struct pkv_pool {
   int sm_count;
   int32_t* d_err;
   int launch_flags;  // PKV_LAUNCH_* bits applied to this pool's kernel launches
+  uint32_t* d_slot_bits;  // pkv_fill's race check: one bit per slot, allocated with the flag
   CUtensorMap tmap;  // 2-D view of the pool: rows of 64 BF16, one 256-row box per page
 };
 
@@ -161,6 +162,7 @@ int pkv_pool_destroy(pkv_pool* pool) {
   cudaSetDevice(pool->device);
   cudaError_t e = cudaDeviceSynchronize();
   cudaFree(pool->d_err);
+  cudaFree(pool->d_slot_bits);
   if (pool->owns_data) cudaFree(pool->data);
   if (prev >= 0) cudaSetDevice(prev);
   delete pool;
@@ -204,6 +206,13 @@ int pkv_fill(pkv_pool* pool, const int32_t* block_tables, const int32_t* cu_toke
     return PKV_ERR_INVALID_ARG;
   // positions are int32 on the device
   if (static_cast<int64_t>(max_blocks) * pkv::kTokens > 2147483647) return PKV_ERR_UNSUPPORTED;
+  if (pool->launch_flags & PKV_LAUNCH_CHECK_APPENDS) {
+    s = from_cuda(pkv::launch_fill_check(layer_slab(block_tables, layer, batch, max_blocks),
+                                         cu_tokens, start_pos, pool->d_slot_bits, pool->d_err,
+                                         batch, max_blocks, pool->num_pages, total_tokens,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+    if (s != PKV_OK) return s;
+  }
   return from_cuda(pkv::launch_fill(
       reinterpret_cast<const __nv_bfloat16*>(k_src), reinterpret_cast<const __nv_bfloat16*>(v_src),
       static_cast<__nv_bfloat16*>(pool->data), layer_slab(block_tables, layer, batch, max_blocks),
@@ -218,6 +227,17 @@ int pkv_pool_set_launch_flags(pkv_pool* pool, int32_t flags) {
   if ((flags & PKV_LAUNCH_EARLY_TABLES) && !(flags & PKV_LAUNCH_PDL)) return PKV_ERR_INVALID_ARG;
   if ((flags & PKV_LAUNCH_EARLY_PAGES) && !(flags & PKV_LAUNCH_EARLY_TABLES))
     return PKV_ERR_INVALID_ARG;
+  if ((flags & PKV_LAUNCH_CHECK_APPENDS) && !pool->d_slot_bits) {
+    // pkv_fill's check needs a slot bitmap: allocated once, here, not in the calls
+    int prev = -1;
+    cudaGetDevice(&prev);
+    cudaSetDevice(pool->device);
+    void* bits = nullptr;
+    const cudaError_t e = cudaMalloc(&bits, pkv::fill_check_bitmap_bytes(pool->num_pages));
+    if (prev >= 0) cudaSetDevice(prev);
+    if (e != cudaSuccess) return from_cuda(e, "pkv_pool_set_launch_flags: cudaMalloc(slot bitmap)");
+    pool->d_slot_bits = static_cast<uint32_t*>(bits);
+  }
   pool->launch_flags = flags;
   return PKV_OK;
 }

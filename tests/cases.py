@@ -95,3 +95,23 @@ APPEND_CONFLICT_CASES = [
     # three writers, two of them on (1,15); the third on (1,0) is read by both
     ("three writers", [[1, 0], [0, 1], [2, 1]], [16, 32, 17], True, True),
 ]
+
+
+# Hand-worked fill-race cases: (name, block-table rows [batch][max_blocks],
+# tokens per sequence, start positions, race), over APPEND_CASE_PAGES pages.
+# Token i of sequence b goes to slot (start+i) % 16 of page row[(start+i) // 16].
+FILL_CONFLICT_CASES = [
+    ("disjoint pages", [[0, 1], [2, 3]], [20, 16], [0, 0], False),
+    # both write slots 2..3 of page 5
+    ("overlapping positions on one page", [[5, 0], [5, 1]], [4, 2], [0, 2], True),
+    # slots 0..3 and 4..7 of page 5
+    ("one page, disjoint slots", [[5, 0], [5, 1]], [4, 4], [0, 4], False),
+    # positions 0 and 16 both land on slot 0 of page 3
+    ("page named twice by one table", [[3, 3]], [17], [0], True),
+    ("page named twice, positions apart", [[3, 3]], [8], [12], False),
+    # both name page 99, outside the pool: neither writes
+    ("writes outside the pool", [[99, 0], [99, 0]], [3, 3], [0, 0], False),
+    # sequence 1 starts beyond its table: skipped, so its overlap does not count
+    ("skipped sequence", [[4, 0], [4, 1]], [5, 5], [0, 30], False),
+    ("empty sequences", [[2, 0], [2, 0], [2, 1]], [0, 0, 3], [0, 0, 0], False),
+]
