@@ -11,7 +11,7 @@ fragmented block tables, 16 layers).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--kernel auto|simt|mma] [--unfused]
-                    [--queries 1..8] [--out-dtype f32|bf16] [--early-pages]
+                    [--queries 1..8] [--out-dtype f32|bf16] [--no-early-pages]
                     [--grid CTAS] [--no-pdl] [--no-fill] [--no-cpu-baseline]
                     [--e2e-steps N] [--cpu-seconds S] [--reference-seconds S]
 
@@ -359,10 +359,9 @@ def run_ours(args, rank, world, local_rank):
         # No kernel of the step writes the lengths or the block tables.  With
         # no separate append, the kernel before each decode (the previous
         # layer's decode or merge) writes no page that decode reads, so its
-        # first page loads may start early too (--early-pages; measured: 2 %
-        # faster on llama1b_b16, no gain on the batch-64 mix).
+        # first page loads start early too (--no-early-pages turns that off).
         flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES
-        if (fused or args.queries > 1) and args.early_pages:
+        if (fused or args.queries > 1) and not args.no_early_pages:
             flags |= pkv.LAUNCH_EARLY_PAGES
         r.pool.set_launch_flags(flags)
     stream = torch.cuda.Stream(device)
@@ -724,8 +723,8 @@ def main():
                     help="oracle time the --impl reference run spends in its timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fill", action="store_true", help="skip the prefill fill timing")
-    ap.add_argument("--early-pages", action="store_true",
-                    help="start the first page loads before the preceding kernel ends")
+    ap.add_argument("--no-early-pages", action="store_true",
+                    help="wait for the preceding kernel before the first page loads")
     ap.add_argument("--queries", type=int, default=1, choices=range(1, 9),
                     help="queries per sequence (> 1: causal among them, decode only)")
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])

@@ -653,9 +653,10 @@ __device__ __forceinline__ OutRowsT<kBf16> out_rows(const DecodeArgs& a, int b, 
 // otherwise (M, S, O) is written as one partial record at `out`.  Pieces are taken 32 at a time
 // (running max rescaled between groups, a fixed order): lane s reads m and l
 // of piece s, and every lane accumulates dims 2*lane, 2*lane+1 of the 4 heads
-// with the loads of kMergeBatch pieces in flight.  kShared: P lives in shared
-// memory (plain loads) instead of global memory (L2 loads).
-constexpr int kMergeBatch = 8;
+// with the loads of kMergeBatch pieces in flight (4: the merge kernel's
+// register cap leaves no room for 8 without spilling).  kShared: P lives in
+// shared memory (plain loads) instead of global memory (L2 loads).
+constexpr int kMergeBatch = 4;
 
 template <bool kShared>
 __device__ __forceinline__ float4 ld4(const float* p) {
@@ -833,8 +834,7 @@ struct SmemPlan {
 };
 
 template <class C>
-__global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
-    decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+__device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const DecodeArgs& a) {
   constexpr int kS = C::kStages;
   using L = SmemPlan<C>;
   extern __shared__ uint8_t smem_raw[];
@@ -1054,6 +1054,25 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   }
 }
 
+template <class C>
+__global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+  decode_body<C>(tmap, a);
+}
+
+// The one-query tensor-core variant needs no more than 88 registers per
+// thread without spilling.  Capped there, its two CTAs per SM leave 20,480
+// of the SM's 65,536 registers free: room for one merge CTA (256 threads at
+// the merge kernel's 80) beside them.  A merge CTA waiting for its decode
+// grid then no longer keeps the next layer's decode CTAs off its SM, so
+// that decode's first page loads (PKV_LAUNCH_EARLY_PAGES) overlap the merge.
+constexpr int kQ1Regs = 88;
+
+__global__ void __maxnreg__(kQ1Regs)
+    decode_kernel_q1(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+  decode_body<MmaComputeT<1, true>>(tmap, a);
+}
+
 // ---------------------------------------------------------------------------
 // Split-KV merge: one CTA per (kv head g, sequence b) unit that decode split
 // into K > 1 pieces.  The split is recomputed here from the lengths (an
@@ -1065,8 +1084,10 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
 // ---------------------------------------------------------------------------
 constexpr int kMergeWarps = 8;
 
+// Three CTAs' worth of registers per SM (at most 85 per thread, 80 used):
+// one merge CTA fits beside two one-query decode CTAs (see decode_kernel_q1).
 template <int kNq, bool kBf16>   // kNq: queries per sequence, 0 = read from the arguments
-__global__ void __launch_bounds__(kMergeWarps * 32)
+__global__ void __launch_bounds__(kMergeWarps * 32, 3)
     merge_kernel(const DecodeArgs a, int32_t decode_grid) {
   __shared__ __align__(16) float s_part[kMergeWarps][kPartialFloats];
   __shared__ int32_t s_sum[2][kMergeWarps];
@@ -1130,9 +1151,18 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
 
 // ---------------------------------------------------------------- host side --
 
+// The kernel that runs compute type C.
+template <class C>
+static auto decode_fn() {
+  if constexpr (std::is_same_v<C, MmaComputeT<1, true>>)
+    return &decode_kernel_q1;
+  else
+    return &decode_kernel<C>;
+}
+
 template <class C>
 static const void* kernel_ptr() {
-  return reinterpret_cast<const void*>(&decode_kernel<C>);
+  return reinterpret_cast<const void*>(decode_fn<C>());
 }
 
 // Tensor-core variants by queries per sequence: 1 (its own, fastest),
@@ -1231,7 +1261,7 @@ static cudaError_t launch_one(const DecodePlan& plan, const CUtensorMap& tmap, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<C>, tmap, a);
+  return cudaLaunchKernelEx(&cfg, decode_fn<C>(), tmap, a);
 }
 
 cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const DecodeArgs& a,
