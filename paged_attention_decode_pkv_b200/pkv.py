@@ -205,7 +205,11 @@ class Pool:
             pass
 
     def set_launch_flags(self, flags: int):
-        """PKV_LAUNCH_* bits for this pool's later kernel launches."""
+        """PKV_LAUNCH_* bits for this pool's later kernel launches (see
+        pkv_pool_set_launch_flags in include/pkv.h).  LAUNCH_CHECK_APPENDS
+        makes append, fill and the fused calls report racing writes as
+        ERR_APPEND_CONFLICT through get_device_error; setting it allocates the
+        pool's slot bitmap once."""
         _check(lib.pkv_pool_set_launch_flags(self.handle, int(flags)), "pkv_pool_set_launch_flags")
 
     def workspace_bytes(self, batch: int, kernel: int = KERNEL_AUTO, grid_ctas: int = 0) -> int:
