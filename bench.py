@@ -633,6 +633,18 @@ def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None, max_la
     return done * w.batch, secs, threads, done
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w, pool_t, max_seconds):
     q, s, thr, layers = oracle_sample(w, pool_t, max_seconds, max_layers=4096)
     q1, s1, _, layers1 = oracle_sample(w, pool_t, max_seconds / 4, max_layers=4096, threads=1)
@@ -640,6 +652,7 @@ def cpu_baseline(w, pool_t, max_seconds):
             "sample": "%d whole-layer append+decode(s) of step 1, cycling over the %d layers "
                       "(%d sequences each), %.1f s of FP64 oracle work" %
                       (layers, w.num_layers, w.batch, s),
+            "cpu_model": cpu_model(),
             "single_core_value": q1 / s1,
             "single_core_sample": "%d whole-layer append+decode(s) on 1 thread, %.1f s" %
                                   (layers1, s1)}
@@ -702,7 +715,7 @@ def run_reference(args, rank, world, local_rank):
         "config": {"workload": w.name, "description": w.description, "batch": B,
                    "layers": nl, "sample": sample},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
