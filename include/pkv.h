@@ -141,18 +141,28 @@ PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
  * only launch latency is hidden.  Also valid under CUDA graph capture.
  * PKV_LAUNCH_EARLY_TABLES (only together with PKV_LAUNCH_PDL) lets decode
  * read seq_lens and the block tables -- never q, the pool or the outputs --
- * before the preceding kernel of the stream has finished, so its set-up
- * overlaps that kernel; the caller guarantees that the kernel launched just
- * before a decode does not write seq_lens or the block tables (an append,
- * which only reads them, is fine).
+ * before the preceding kernels of the stream have finished, so its set-up
+ * overlaps them.  Every kernel of this library lets the next launch start
+ * early, so "preceding kernels" means every earlier kernel of the stream
+ * that may still be running, not only the one launched just before (the
+ * previous decode can still run beside its split-KV merge, for instance).
+ * The caller guarantees that none of them writes seq_lens or the block
+ * tables (an append or a decode, which only read them, is fine).
  * PKV_LAUNCH_EARLY_PAGES (only together with both) lets decode also start
  * loading the first pages of its range -- the KV of tokens already in the
- * cache -- before that kernel has finished, so their memory latency overlaps
- * it; q, the new token's rows and the outputs still wait.  The caller
- * guarantees that the kernel launched just before a decode does not write
- * the pool pages it reads: true when that kernel is the previous layer's
- * decode or merge, or a projection that writes q; false when it is a
- * pkv_append or pkv_fill into this layer (use the fused call instead).
+ * cache -- before those kernels have finished, so their memory latency
+ * overlaps them; q, the new token's rows and the outputs still wait.  These
+ * early loads never touch a sequence's last two pages: that is where an
+ * append or a fused append + decode of the same layer writes the newest
+ * tokens (one per step, so the pages of the preceding 16 steps' tokens), so
+ * chains of fused calls, or of pkv_append then decode, on one layer are
+ * safe, repeated steps of a one-layer model included.  The caller
+ * guarantees that no other pool page a decode reads is written by a kernel
+ * that may still be running: true for the decodes and merges of other
+ * layers and for a projection that writes q; false for a pkv_fill into this
+ * layer's pages (its tokens can land in any page) or for a caller kernel
+ * that writes pages, unless that kernel completes before decode starts
+ * (launch decode without this flag after it).
  * PKV_LAUNCH_CHECK_APPENDS makes pkv_append, pkv_fill and the fused calls
  * (paged_attention_decode_append[_ex], pkv_decode with k_new) first launch a
  * check, on the same stream, that records PKV_ERR_APPEND_CONFLICT when the
@@ -410,10 +420,14 @@ PKV_API int pkv_gather(const pkv_pool *pool, const int32_t *block_tables, const 
  * scratch area of PKV_NOALLOC_SCRATCH_BYTES that the library keeps in every
  * GPU's memory from load until process exit.  It allocates nothing.
  *  - Limit: returns PKV_ERR_TOO_LARGE (nothing launched) when the batch
- *    needs more scratch than that (pkv_decode_workspace_bytes > limit); on a
- *    B200 with the default grid this allows about 1,600 sequences.
- *  - The first call on a device looks up the scratch's device address
- *    (cudaGetSymbolAddress, with the pool's device current); make that first
+ *    needs more scratch than that, i.e. when pkv_decode_workspace_bytes for
+ *    this pool and batch (the exact check) exceeds it.  That size is
+ *    (batch + grid) * 8 * 1056 bytes, grid being the decode kernel's CTAs
+ *    (SM count x CTAs per SM: 296 on a B200 while the batch is small enough
+ *    for two CTAs per SM), so a B200 takes up to 1,689 sequences.
+ *  - Every call looks up the scratch's device address (cudaGetSymbolAddress,
+ *    with the pool's device current; nothing is allocated).  The first
+ *    lookup on a device may load the library's device code: make the first
  *    call before any stream capture.
  *  - All calls on one device share the one scratch area, which keeps the
  *    last call's contents; nothing in it has to start at zero.  Calls whose

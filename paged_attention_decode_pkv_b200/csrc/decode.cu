@@ -799,8 +799,12 @@ __device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a,
 }
 
 // Producer-side description of page f (this lane's slot of a 32-page batch):
-// physical page, and (sequence << 2) | (last page of the sequence << 1) |
-// starts-a-sequence-in-this-range.
+// physical page, and (sequence << kInfoSeqShift) | kInfoRecent (one of the
+// sequence's last two pages) | kInfoLast (its last page) | kInfoStart
+// (starts a sequence in this range).
+constexpr int32_t kInfoStart = 1, kInfoLast = 2, kInfoRecent = 4;
+constexpr int kInfoSeqShift = 3;
+
 __device__ __forceinline__ void load_page_batch(const DecodeArgs& a, const int32_t* s_pfx,
                                                 int32_t f, int32_t f_begin, int32_t f_end,
                                                 int32_t& phys, int32_t& info) {
@@ -810,8 +814,9 @@ __device__ __forceinline__ void load_page_batch(const DecodeArgs& a, const int32
     int b, j;
     locate(s_pfx, a.batch, f, b, j);
     phys = __ldg(a.bt + static_cast<int64_t>(b) * a.max_blocks + j);
-    info = (b << 2) | ((j == s_pfx[b + 1] - s_pfx[b] - 1) ? 2 : 0) |
-           ((j == 0 || f == f_begin) ? 1 : 0);
+    const int np = s_pfx[b + 1] - s_pfx[b];
+    info = (b << kInfoSeqShift) | (j >= np - 2 ? kInfoRecent : 0) |
+           (j == np - 1 ? kInfoLast : 0) | ((j == 0 || f == f_begin) ? kInfoStart : 0);
   }
 }
 
@@ -863,11 +868,12 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
     fence_mbar_init();
   }
   // With kLaunchEarlyTables the lengths and block tables are read before the
-  // preceding kernel of the stream has finished (the caller guarantees that
-  // kernel does not write them); q, the pool and the outputs only after.
-  // With kLaunchEarlyPages as well, the first kS pages' loads are issued
-  // before that kernel has finished too (the caller guarantees it does not
-  // write those pages); their query rows and new-token rows only after.
+  // preceding kernels of the stream have finished (the caller guarantees
+  // they do not write them); q, the pool and the outputs only after.  With
+  // kLaunchEarlyPages as well, the loads of the first kS pages go out before
+  // then too, except for pages among a sequence's last two (see below; the
+  // caller guarantees nothing still running writes the others); their query
+  // rows and new-token rows only after.
   const bool early = (a.flags & kLaunchEarlyTables) != 0;
   const bool early_pages = early && (a.flags & kLaunchEarlyPages) != 0;
   if (!early) pdl_wait();
@@ -920,9 +926,9 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
       const uint32_t bar = full + 8 * st;
       const uint32_t dst = base + L::stages + st * L::kStageBytes;
       const bool ok = static_cast<uint32_t>(phys) < static_cast<uint32_t>(a.num_pages);
-      const bool start = info & 1;
-      const bool append = fused && (info & 2);
-      const int64_t seq = info >> 2;
+      const bool start = info & kInfoStart;
+      const bool append = fused && (info & kInfoLast);
+      const int64_t seq = info >> kInfoSeqShift;
       const uint32_t rows = (start ? nq * kQRowsBytes : 0) + (append ? kNewRowsBytes : 0);
       if (part & kIssuePage) {
         s_flags[st] = ok ? 0 : 1;
@@ -948,8 +954,18 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
       }
     }
   };
+  // Early loads skip a sequence's last two pages: a kernel still running
+  // before this one may write the newest tokens there (a fused decode or an
+  // append of this layer at an earlier step: one token per step, so the
+  // last 16 steps' tokens lie in those two pages).  early_mask: pages r < kS
+  // whose page part went out early.
+  uint32_t early_mask = 0;
   if (warp == 0 && early_pages)
-    for (int r = 0; r < n && r < kS; ++r) issue(r, kIssuePage);
+    for (int r = 0; r < n && r < kS; ++r)
+      if (!(__shfl_sync(kFull, cur_info, r & 31) & kInfoRecent)) {
+        issue(r, kIssuePage);
+        early_mask |= 1u << r;
+      }
   if (early) pdl_wait();
 
   // empty (or invalid) sequences: zero output rows, once across the grid
@@ -958,7 +974,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
   if (n <= 0) return;
   if (warp == 0)
     for (int r = 0; r < n && r < kS; ++r)
-      issue(r, early_pages ? kIssueRows : kIssuePage | kIssueRows);
+      issue(r, (early_mask >> r) & 1u ? kIssueRows : kIssuePage | kIssueRows);
   // After a timed-out wait: wait (bounded) for the copies still in flight
   // into this CTA's stages, pages k0 .. issued-1, before the CTA exits.
   auto drain = [&](int k0) {

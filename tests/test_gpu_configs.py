@@ -86,13 +86,17 @@ def test_llama1b_batch16_all_layers(kernel):
     _check(got, want, gp, hp)
 
 
+def _bench_flags():
+    import bench
+    return bench.launch_flags(pkv)
+
+
 @pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("fused", [False, True])
 def test_continuous_batching_batch64(kernel, fused):
     w = W.continuous_batching()
-    flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES   # as the benchmark launches it
     got, want, gp, hp, _ = _run(w, kernel, sample_layers=[0, 15],
-                                sample_steps=[1, w.num_steps], flags=flags, fused=fused)
+                                sample_steps=[1, w.num_steps], flags=_bench_flags(), fused=fused)
     _check(got, want, gp, hp)
 
 
@@ -100,16 +104,9 @@ def test_continuous_batching_batch64(kernel, fused):
 @pytest.mark.parametrize("fused", [False, True])
 def test_long_context_batch4(kernel, fused):
     w = W.long_context()
-    flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES if fused else 0
+    flags = _bench_flags() if fused else 0
     got, want, gp, hp, _ = _run(w, kernel, sample_layers=[0], sample_steps=[1], flags=flags,
                                 fused=fused)
-    _check(got, want, gp, hp)
-
-
-def test_llama1b_batch16_fused_as_benchmarked():
-    w = W.llama1b()
-    got, want, gp, hp, _ = _run(w, pkv.KERNEL_AUTO, sample_layers=[0, 7, 15], sample_steps=[1],
-                                flags=pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES, fused=True)
     _check(got, want, gp, hp)
 
 
@@ -153,3 +150,77 @@ def test_stress_batch256_sampled():
     # nothing else in the pool changed
     after = _slot_checksums(pool_t)
     assert torch.equal(before["cs"][~touched], after[~touched])
+
+
+# ---------------------------------------------------------------------------
+# The benchmarked launch itself: bench.py's Runner (one CUDA graph per step of
+# 16 fused append + decode calls plus their merges), with bench.py's launch
+# flags (programmatic dependent launch, tables and first pages read before
+# the preceding kernels end), replayed step after step as the benchmark
+# replays it.  The only difference from the benchmark: before each step's
+# replay the step's own inputs are copied into the graphs' input buffers
+# (the benchmark reuses one set), so every step appends and attends to fresh
+# tokens that the oracle also sees.
+
+def _run_as_benchmarked(w, sample_layers, sample_steps, rows=None):
+    import bench
+    dev = torch.device("cuda", 0)
+    rows = np.arange(w.batch) if rows is None else np.asarray(rows)
+    r = bench.Runner(w, dev, pkv.KERNEL_AUTO, fused=True)
+    flags = bench.launch_flags(pkv)
+    assert flags == pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES | pkv.LAUNCH_EARLY_PAGES
+    r.pool.set_launch_flags(flags)
+    host_pool, host_bt = W.compact_pages(w, r.pool_t, rows, sample_layers)
+    host_pool = host_pool.reshape(-1, 2, 8, 16, 64).copy()
+    stream = torch.cuda.Stream(dev)
+    r.capture(stream)
+    got, want = {}, {}
+    for step in range(1, w.num_steps + 1):
+        sl_np = r.lens_np[step - 1]
+        assert np.array_equal(sl_np, w.seq_lens(step))
+        ins = [W.step_inputs(w, step, l, dev) for l in range(w.num_layers)]
+        for l, (q, k, v) in enumerate(ins):
+            r.q[l].copy_(q)
+            r.k[l].copy_(k)
+            r.v[l].copy_(v)
+        r.replay(step - 1)
+        for layer in sample_layers:
+            q, k, v = ins[layer]
+            _append_rows(host_pool, host_bt, sl_np, bits(k), bits(v), layer, rows)
+            if step in sample_steps:
+                got[(step, layer)] = r.out[layer][rows].cpu().numpy().astype(np.float64)
+                want[(step, layer)] = oracle.decode(bits(q), host_pool, host_bt, sl_np, layer,
+                                                    w.scale, rows=rows)[rows]
+    torch.cuda.synchronize()
+    assert pkv.get_device_error(r.pool) == 0
+    gpu_pages, _ = W.compact_pages(w, r.pool_t, rows, sample_layers)
+    pages = gpu_pages.reshape(host_pool.shape)
+    r.close()
+    return got, want, pages, host_pool
+
+
+def test_continuous_batching_batch64_as_benchmarked():
+    w = W.continuous_batching()
+    got, want, gp, hp = _run_as_benchmarked(w, sample_layers=[0, 7, 15],
+                                            sample_steps=[1, 2, 8, 15, 16])
+    _check(got, want, gp, hp)
+
+
+def test_llama1b_batch16_as_benchmarked():
+    w = W.llama1b()
+    got, want, gp, hp = _run_as_benchmarked(w, sample_layers=list(range(16)), sample_steps=[1])
+    _check(got, want, gp, hp)
+
+
+def test_long_context_batch4_as_benchmarked():
+    w = W.long_context()
+    got, want, gp, hp = _run_as_benchmarked(w, sample_layers=[0], sample_steps=[1])
+    _check(got, want, gp, hp)
+
+
+def test_stress_batch256_as_benchmarked_sampled():
+    w = W.stress()
+    rows = [0, 37, 64, 101, 128, 199, 230, 255]
+    got, want, gp, hp = _run_as_benchmarked(w, sample_layers=[0, 15],
+                                            sample_steps=[1, 2, 25, w.num_steps], rows=rows)
+    _check(got, want, gp, hp)

@@ -89,34 +89,54 @@ def test_fused_split_patterns_bitwise_equal_to_two_calls(kernel, grid, min_chunk
         assert pkv.get_device_error(fused.pool) == 0
 
 
+EARLY_ALL = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES | pkv.LAUNCH_EARLY_PAGES
+
+
 @pytest.mark.parametrize("kernel", KERNELS)
-@pytest.mark.parametrize("flags", [pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES,
-                                   pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES |
-                                   pkv.LAUNCH_EARLY_PAGES])
-def test_fused_repeated_steps_with_pdl(kernel, flags):
-    # several decode steps: lengths grow by one, each step appends and attends;
-    # with early pages each launch starts loading its first pages while the
-    # previous step's kernels run (they write other slots only)
-    lens0 = np.array([40, 1, 77, 15, 300], np.int32)
+@pytest.mark.parametrize("flags", [pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES, EARLY_ALL])
+@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("lens0,grid", [([40, 1, 77, 15, 300], 0),
+                                        ([40, 1, 77, 15, 300], 3),
+                                        (list(range(1, 33)) + [200, 31, 17], 0)])
+def test_repeated_steps_on_one_layer_with_pdl(kernel, flags, fused, lens0, grid):
+    # Steps of a one-layer model: lengths grow by one, each step appends the
+    # new token (fused, or pkv_append then decode) and attends to it.  With
+    # programmatic launch a step's decode may start while the previous
+    # step's kernels still run -- and with early pages load pages before
+    # they end -- so the pages the previous steps append into must not be
+    # loaded early.  Every step is checked against the oracle, and the pool
+    # bit for bit at the end.  Lengths cross page boundaries during the 20
+    # steps, and the many short sequences put CTA ranges' first pages on
+    # sequences' last pages.
+    lens0 = np.array(lens0, np.int32)
     steps = 20
-    c = make_case(list(lens0 + steps), seed=31, spare_pages=3)
+    B = lens0.size
+    c = make_case(list(lens0 + steps), seed=31 + B, spare_pages=3)
     g = GpuCase(c)
     g.pool.set_launch_flags(flags)
     host = c["pool"].copy()
     rng = np.random.default_rng(5)
     from tests.cases import bf16_bits
+    outs, wants = [], []
     for s in range(1, steps + 1):
         sl = lens0 + s
-        k = bf16_bits(rng.standard_normal((5, 8, 64)))
-        v = bf16_bits(rng.standard_normal((5, 8, 64)))
-        out = pkv.decode_append(g.q, u16_to_bf16(k), u16_to_bf16(v), g.pool, g.bt, to_dev(sl), 0,
-                                0.125, kernel=kernel)
+        k = bf16_bits(rng.standard_normal((B, 8, 64)))
+        v = bf16_bits(rng.standard_normal((B, 8, 64)))
+        sl_d = to_dev(sl)
+        if fused:
+            out = pkv.decode_append(g.q, u16_to_bf16(k), u16_to_bf16(v), g.pool, g.bt, sl_d, 0,
+                                    0.125, kernel=kernel, grid_ctas=grid)
+        else:
+            pkv.append(g.pool, g.bt, sl_d, u16_to_bf16(k), u16_to_bf16(v), 0)
+            out = pkv.decode(g.q, g.pool, g.bt, sl_d, 0, 0.125, kernel=kernel, grid_ctas=grid)
         oracle.append(host, c["bt"], sl, k, v, 0)
+        outs.append(out)
+        wants.append(oracle.decode(c["q"], host, c["bt"], sl, 0, 0.125))
     torch.cuda.synchronize()
     assert pkv.get_device_error(g.pool) == 0
     assert np.array_equal(bits(g.pool_t).reshape(host.shape), host)
-    want = oracle.decode(c["q"], host, c["bt"], lens0 + steps, 0, 0.125)
-    assert max_err(out.cpu().numpy().astype(np.float64), want) <= ATOL
+    for s, (out, want) in enumerate(zip(outs, wants), 1):
+        assert max_err(out.cpu().numpy().astype(np.float64), want) <= ATOL, s
 
 
 def test_fused_bad_last_page_is_reported_and_not_written():
