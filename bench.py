@@ -13,26 +13,35 @@ fragmented block tables, 16 layers).
                     [--impl ours|reference] [--kernel auto|simt|mma] [--unfused]
                     [--queries 1..8] [--out-dtype f32|bf16] [--no-early-pages]
                     [--grid CTAS] [--no-pdl] [--no-fill] [--no-cpu-baseline]
+                    [--also W1,W2 | --also none] [--cold-l2] [--clock-seconds S]
                     [--e2e-steps N] [--cpu-seconds S] [--reference-seconds S]
+    python bench.py --table      # every workload and option row, one run
 
 Prints one JSON line (rank 0).  ``value`` is decode-queries/s over all
 ranks, one query being one sequence's 32 query heads at one layer
 (``head_queries_per_s`` counts heads, ``tokens_per_s`` sequences' tokens
 per whole-model step; ``append``, in --unfused runs, the separate append's
-share of a layer).  The
-``roofline`` object reports the decode kernel's algorithmic HBM bytes per
-launch divided by its measured average launch time, against the measured
-HBM copy bandwidth, with the DRAM traffic of the committed ncu capture.
-``e2e`` is the same step with its inputs and outputs crossing from and to
-pinned host memory every step; ``prefill_fill`` the page-fill bandwidth;
+share of a layer).  The ``roofline`` object reports the decode call's
+algorithmic HBM bytes per launch divided by its measured average launch
+time, against the measured HBM copy bandwidth, with the DRAM traffic of the
+committed ncu capture.  ``clocks`` are sampled over the timed steps and a
+following window of at least --clock-seconds of the same graph replays
+(``clocks.window``: that window's own per-launch time).  ``per_workload``
+holds the same measurement for the other workloads the speed target names
+(long context, and the Llama-1B batch with a cold-L2 figure).  ``e2e`` is
+the same step with its inputs and outputs crossing from and to pinned host
+memory every step; ``prefill_fill`` the page-fill bandwidth;
 ``cpu_baseline`` the FP64 oracle on the host cores.  ``--impl reference``
 times the FP64 CPU oracle on the same workload instead (bounded sample per
-step, host cores).
+step, host cores).  ``--table`` measures every workload (hot and cold L2
+for the two whose layer fits in L2) and the multi-query, BF16-output and
+fill rows, and prints them as JSON lines and a markdown table.
 """
 from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -155,7 +164,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.reader = threading.Thread(target=self._read, daemon=True)
             self.reader.start()
@@ -236,6 +245,20 @@ def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
 
 # ---------------------------------------------------------------- our arm --
 
+def launch_flags(pkv, pdl: bool = True, early_pages: bool = True) -> int:
+    """Pool launch flags of the benchmarked step.  No kernel of the step
+    writes the lengths or the block tables, and the only pages a step writes
+    are the sequences' last pages (the appended token), which decode never
+    loads early, so with PDL both early flags hold for the fused and the
+    separate-append step alike."""
+    if not pdl:
+        return 0
+    flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES
+    if early_pages:
+        flags |= pkv.LAUNCH_EARLY_PAGES
+    return flags
+
+
 class Runner:
     """Device-resident state of one workload on one GPU."""
 
@@ -273,6 +296,8 @@ class Runner:
         oshape = (nl, B, 32, 64) if queries == 1 else (nl, B, queries, 32, 64)
         self.out = torch.empty(oshape, dtype=out_dtype, device=device)
         self.ws = self.pool.workspace(B, kernel, grid, queries)
+        self.graphs, self.decode_graphs = [], []
+        self.twins = []
 
     def twin(self, stream):
         """A second set of step inputs and outputs (same pool, tables and
@@ -284,7 +309,9 @@ class Runner:
         t.seq_lens = [x.clone() for x in self.seq_lens]
         t.q, t.k, t.v = self.q.clone(), self.k.clone(), self.v.clone()
         t.out = torch.empty_like(self.out)
+        t.twins = []
         t.capture(stream)
+        self.twins.append(t)
         return t
 
     def launch_step(self, stream, variant, decode_only=False):
@@ -344,135 +371,263 @@ class Runner:
                              self.out.element_size())
         return b + (4096 * self.w.batch if self.fused else 0)
 
+    def mean_decode_bytes(self, start, n):
+        """Mean of decode_bytes(i) over steps start .. start + n - 1."""
+        per = [self.decode_bytes(v) for v in range(self.w.num_steps)]
+        full, rem = divmod(n, len(per))
+        tot = full * sum(per) + sum(per[(start + j) % len(per)] for j in range(rem))
+        return tot / n
 
-def run_ours(args, rank, world, local_rank):
+    def kernels_per_layer(self, decode_only=False):
+        """Kernels one layer of a step launches: the decode kernel and the
+        split-KV merge, plus the separate append unless fused."""
+        return 2 + (0 if self.fused or decode_only or self.queries > 1 else 1)
+
+    def close(self):
+        """Release the graphs (they hold this library's kernel nodes), the
+        twins' graphs and the pool, device synchronised, before anything
+        they reference goes away."""
+        torch.cuda.synchronize(self.device)
+        for t in self.twins:
+            t.graphs, t.decode_graphs = [], []
+        self.twins = []
+        self.graphs, self.decode_graphs = [], []
+        self.pool.close()
+
+
+def _events():
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def _replays(r: Runner, stream, steps, decode_only=False, start=0):
+    """CUDA-event time (ms) of `steps` back-to-back step replays on `stream`."""
+    e0, e1 = _events()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(start, start + steps):
+            (r.replay_decodes if decode_only else r.replay)(i)
+        e1.record(stream)
+    return e0, e1
+
+
+def _cold_replays(r: Runner, stream, steps, decode_only=False):
+    """Per-step CUDA-event times (ms) with L2 flushed before every step: a
+    buffer twice the L2 size is written between replays, outside the
+    timed events."""
+    l2 = torch.cuda.get_device_properties(r.device).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=r.device)
+    pairs = []
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = _events()
+            e0.record(stream)
+            (r.replay_decodes if decode_only else r.replay)(i)
+            e1.record(stream)
+            pairs.append((e0, e1))
+    stream.synchronize()
+    del flush
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def measure(args, name, device, rank, world, local_rank, *, full=False, cold=False,
+            cpu_seconds=0.0, cpu_rows=None, queries=None, out_dtype=None, kernel=None):
+    """Set up one workload and time its step the way the benchmark line
+    reports it.  Every rank runs the same collectives in the same order.
+    Returns the workload's record (rank 0) or None."""
     from paged_attention_decode_pkv_b200 import pkv
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    kernel = {"auto": pkv.KERNEL_AUTO, "simt": pkv.KERNEL_SIMT, "mma": pkv.KERNEL_MMA}[args.kernel]
-    w = workload_for_rank(args.workload, rank)
-    fused = not args.unfused and args.queries == 1
-    out_dtype = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
-    r = Runner(w, device, kernel, fused, args.queries, out_dtype, args.grid)
-    flags = 0
-    if not args.no_pdl:
-        # No kernel of the step writes the lengths or the block tables.  With
-        # no separate append, the kernel before each decode (the previous
-        # layer's decode or merge) writes no page that decode reads, so its
-        # first page loads start early too (--no-early-pages turns that off).
-        flags = pkv.LAUNCH_PDL | pkv.LAUNCH_EARLY_TABLES
-        if (fused or args.queries > 1) and not args.no_early_pages:
-            flags |= pkv.LAUNCH_EARLY_PAGES
-        r.pool.set_launch_flags(flags)
+    queries = args.queries if queries is None else queries
+    out_dtype = args.out_dtype if out_dtype is None else out_dtype
+    kname = args.kernel if kernel is None else kernel
+    kern = {"auto": pkv.KERNEL_AUTO, "simt": pkv.KERNEL_SIMT, "mma": pkv.KERNEL_MMA}[kname]
+    w = workload_for_rank(name, rank)
+    fused = not args.unfused and queries == 1
+    tdtype = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+    r = Runner(w, device, kern, fused, queries, tdtype, args.grid)
+    flags = launch_flags(pkv, pdl=not args.no_pdl, early_pages=not args.no_early_pages)
+    r.pool.set_launch_flags(flags)
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             r.launch_step(stream, i % w.num_steps)
     stream.synchronize()
-    assert pkv.get_device_error(r.pool, stream) == 0
+    if pkv.get_device_error(r.pool, stream) != 0:
+        raise RuntimeError("device error in the warm-up steps of %s" % name)
     r.capture(stream)
     for i in range(max(args.warmup, w.num_steps)):
         r.replay(i)
+        if not fused:
+            r.replay_decodes(i)
     torch.cuda.synchronize()
 
     # ---- timed region: (A) K full steps; unfused only, then (B) the decodes
-    # of K steps alone, back to back, for the decode kernel's launch duration
-    # (fused, a step is nothing but the decode launches, so (A) gives it)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if not fused:
-        for i in range(max(args.warmup, w.num_steps)):
-            r.replay_decodes(i)
+    # of K steps alone, back to back, for the decode call's launch duration
+    # (fused, a step is nothing but the decode calls, so (A) gives it).  The
+    # clock sampler keeps running over a window of at least clock_seconds of
+    # the same full-step replays right after, so that its record has samples
+    # however short the timed region is.
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
-        with torch.cuda.stream(stream):
-            t0.record(stream)
-            for i in range(args.steps):
-                r.replay(i)
-            t1.record(stream)
-            if not fused:
-                d0.record(stream)
-                for i in range(args.steps):
-                    r.replay_decodes(i)
-                d1.record(stream)
+        t0, t1 = _replays(r, stream, args.steps)
+        if not fused:
+            d0, d1 = _replays(r, stream, args.steps, decode_only=True)
         stream.synchronize()
-        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1)
+        n_win = max(1, int(math.ceil(args.clock_seconds * 1e3 / max(ms / args.steps, 1e-3))))
+        n_win = min(n_win, 2_000_000)
+        w0, w1 = _replays(r, stream, n_win, start=args.steps)
+        stream.synchronize()
     barrier()
-    ms = t0.elapsed_time(t1)
-    dec_launches = args.steps * w.num_layers
-    dec_ms = t0.elapsed_time(t1) if fused else d0.elapsed_time(d1)
-    avg_dec_s = max_over_ranks(dec_ms, device) / dec_launches / 1e3
-    avg_bytes = sum(r.decode_bytes(i) for i in range(args.steps)) / args.steps
+    torch.cuda.synchronize()
+    layers = w.num_layers
+    dec_launches = args.steps * layers
+    dec_ms = ms if fused else d0.elapsed_time(d1)
+    win_ms = w0.elapsed_time(w1)
     err = pkv.get_device_error(r.pool, stream)
     if err != 0:
-        raise RuntimeError("device error during timed region: %s" % pkv.status_string(err))
+        raise RuntimeError("device error during the timed region: %s" % pkv.status_string(err))
     ms = max_over_ranks(ms, device)
-    value = whole_job_rate(args.steps * w.num_layers * w.batch * r.queries, world, ms)
+    avg_dec_s = max_over_ranks(dec_ms, device) / dec_launches / 1e3
+    units = layers * w.batch * r.queries   # decode-queries per step
+    value = whole_job_rate(args.steps * units, world, ms)
+    avg_bytes = r.mean_decode_bytes(0, args.steps)
+    win_bytes = r.mean_decode_bytes(args.steps, n_win)
 
-    # ---- end to end through the public API from pinned host buffers
-    e2e = run_e2e(r, stream, min(args.steps, args.e2e_steps), device, world)
+    cold_ms = None
+    if cold:
+        reps = min(args.steps, 50)
+        cold_ms = max_over_ranks(sum(_cold_replays(r, stream, reps, decode_only=not fused)), device)
+        cold_reps = reps
+    append_us = None
+    if not fused and r.queries == 1:
+        append_us = (t0.elapsed_time(t1) - d0.elapsed_time(d1)) / dec_launches * 1e3
 
-    # ---- prefill page fill bandwidth (rewrites the prompt tokens' values)
-    fill = None if args.no_fill else run_fill(r, stream, min(args.steps, 50), device)
-
+    e2e = run_e2e(r, stream, args.e2e_steps, device, world) if full else None
+    fill = run_fill(r, stream, min(args.steps, 50), device) if full and not args.no_fill \
+        else None
+    cpu = None
+    if cpu_seconds > 0 and world == 1 and rank == 0:
+        cpu = cpu_baseline(w, r.pool_t, cpu_seconds, rows=cpu_rows)
+    r.close()
     if rank != 0:
         return None
+
     peak, peak_kind = measured_peaks()
     achieved = avg_bytes / avg_dec_s / 1e9
-    traffic = recorded_traffic(w.name, avg_bytes)
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {
-            "workload": w.name, "description": w.description, "batch": w.batch,
-            "layers": w.num_layers, "pool_pages": w.num_pages,
-            "kv_bytes_per_layer": w.kv_bytes(1), "accumulate": "f32",
-            "kernel": args.kernel, "parallelism": "dp%d (independent replicas)" % world,
-            "queries_per_sequence": r.queries, "out_dtype": args.out_dtype,
-            "launch": "one CUDA graph per step (16 x %s + split merge)%s" %
-                      ("fused append+decode" if fused else
-                       "%d-query decode" % r.queries if r.queries > 1 else "append + decode",
-                       "" if args.no_pdl else ", programmatic dependent launch, tables %sread "
-                                              "before the preceding kernel ends" %
-                       ("and first pages " if flags & pkv.LAUNCH_EARLY_PAGES else "")),
-            "l2": "inputs larger than L2: one step reads %.0f MB of K/V" %
-                  (w.kv_bytes(1) * w.num_layers / 1e6),
-        },
+    win_achieved = win_bytes / (win_ms / (n_win * layers) / 1e3) / 1e9
+    clocks = clk.summary()
+    clocks["window"] = {
+        "what": "sampler running over the %d timed steps and %d more replays of the same "
+                "step graphs right after them" % (args.steps, n_win),
+        "seconds": (ms + win_ms) / 1e3, "replays": n_win,
+        "us_per_launch": win_ms / (n_win * layers) * 1e3,
+        "achieved_gbs": win_achieved, "frac": win_achieved / peak}
+    rec = {
+        "workload": w.name, "description": w.description, "batch": w.batch, "layers": layers,
+        "pool_pages": w.num_pages, "kv_bytes_per_layer": w.kv_bytes(1),
+        "queries_per_sequence": r.queries, "out_dtype": out_dtype, "kernel": kname,
+        "fused": fused, "flags": flags, "steps": args.steps, "ms_per_step": ms / args.steps,
+        "value": value, "unit": UNIT,
+        "decode_queries_per_s": w.batch * r.queries / avg_dec_s,
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+            "frac": achieved / peak, "traffic": recorded_traffic(w.name, avg_bytes)
+            if r.queries == 1 and out_dtype == "f32" else None,
+            "peak_kind": peak_kind,
             "kernel": "decode_kernel%s (+ split-KV merge_kernel)" %
                       (" with fused append" if fused else ""),
             "alg_bytes_per_launch": avg_bytes, "avg_launch_us": avg_dec_s * 1e6,
-            "launches": dec_launches,
-        },
-        "decode_queries_per_s": w.batch * r.queries / avg_dec_s,
-        "head_queries_per_s": value * 32,
-        "tokens_per_s": value / w.num_layers,
-        "e2e": e2e,
-        "prefill_fill": fill,
-        "gpu_launches": (args.steps * w.num_layers * (2 if fused or r.queries > 1 else 3) +
-                         (0 if fused else dec_launches * 2)),
+            "launches": dec_launches},
+        "gpu_launches": args.steps * layers * r.kernels_per_layer() +
+                        (0 if fused else dec_launches * r.kernels_per_layer(decode_only=True)),
         "decode_timing": ("CUDA events around the %d full-step replays (fused append + decode "
                           "+ merge per layer, %d launches)" % (args.steps, dec_launches)
                           if fused else
                           "CUDA events around %d back-to-back replays of the step's decode "
-                          "launches alone (decode + merge per layer, %d launches)" %
+                          "calls alone (decode + merge per layer, %d launches)" %
                           (args.steps, dec_launches)),
-        "clocks": clk.summary(),
+        "clocks": clocks,
+        "kernel_source_sha256": kernel_source_digest(),
     }
-    if not fused and r.queries == 1:
-        # the separate append's share of a layer: full step replays minus the
-        # replays of the same decode + merge launches alone
-        line["append"] = {
-            "kernel": "append_kernel", "us_per_launch":
-                (t0.elapsed_time(t1) - d0.elapsed_time(d1)) / dec_launches * 1e3,
+    if cold_ms is not None:
+        cold_us = cold_ms / (cold_reps * layers) * 1e3
+        cold_ach = avg_bytes / (cold_us / 1e6) / 1e9
+        rec["cold_l2"] = {
+            "us_per_launch": cold_us, "achieved": cold_ach, "frac": cold_ach / peak,
+            "how": "%d steps, each replayed alone after writing 2 x L2 bytes, CUDA events "
+                   "around each replay; per launch = total / (steps x layers)" % cold_reps}
+    if append_us is not None:
+        rec["append"] = {
+            "kernel": "append_kernel", "us_per_launch": append_us,
             "bytes_per_launch": w.batch * (2 * 2048 + 8),
             "how": "unfused step time minus decode + merge time, per layer (PDL-chained)"}
-    if not args.no_cpu_baseline and world == 1:   # the host baseline is taken at N = 1 only
-        line["cpu_baseline"] = cpu_baseline(w, r.pool_t, args.cpu_seconds)
+    if e2e is not None:
+        rec["e2e"] = e2e
+    if fill is not None:
+        rec["prefill_fill"] = fill
+    if cpu is not None:
+        rec["cpu_baseline"] = cpu
+    return rec
+
+
+def run_ours(args, rank, world, local_rank):
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    main = measure(args, args.workload, device, rank, world, local_rank, full=True,
+                   cold=args.cold_l2,
+                   cpu_seconds=0.0 if args.no_cpu_baseline else args.cpu_seconds)
+    others = []
+    for name in args.also:
+        rec = measure(args, name, device, rank, world, local_rank,
+                      cold=name in COLD_WORKLOADS or args.cold_l2,
+                      cpu_seconds=0.0 if args.no_cpu_baseline else min(args.cpu_seconds, 3.0))
+        others.append(rec)
+    if rank != 0:
+        return None
+    m = main
+    line = {
+        "metric": METRIC, "value": m["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": m["workload"], "description": m["description"], "batch": m["batch"],
+            "layers": m["layers"], "pool_pages": m["pool_pages"],
+            "kv_bytes_per_layer": m["kv_bytes_per_layer"], "accumulate": "f32",
+            "kernel": m["kernel"], "parallelism": "dp%d (independent replicas)" % world,
+            "queries_per_sequence": m["queries_per_sequence"], "out_dtype": m["out_dtype"],
+            "launch": "one CUDA graph per step (16 x %s + split merge)%s" %
+                      ("fused append+decode" if m["fused"] else
+                       "%d-query decode" % m["queries_per_sequence"]
+                       if m["queries_per_sequence"] > 1 else "append + decode",
+                       "" if args.no_pdl else ", programmatic dependent launch, tables %sread "
+                                              "before the preceding kernels end" %
+                       ("and first pages " if m["flags"] & 4 else "")),
+            "l2": "inputs larger than L2: one step reads %.0f MB of K/V" %
+                  (m["kv_bytes_per_layer"] * m["layers"] / 1e6),
+        },
+        "roofline": m["roofline"],
+        "decode_queries_per_s": m["decode_queries_per_s"],
+        "head_queries_per_s": m["value"] * 32,
+        "tokens_per_s": m["value"] / m["layers"],
+        "e2e": m.get("e2e"),
+        "prefill_fill": m.get("prefill_fill"),
+        "gpu_launches": m["gpu_launches"],
+        "decode_timing": m["decode_timing"],
+        "clocks": m["clocks"],
+        "kernel_source_sha256": m["kernel_source_sha256"],
+    }
+    for k in ("append", "cold_l2", "cpu_baseline"):
+        if k in m:
+            line[k] = m[k]
+    if others:
+        line["per_workload"] = {
+            o["workload"]: {k: o[k] for k in ("value", "unit", "ms_per_step", "roofline",
+                                              "decode_queries_per_s", "clocks", "cold_l2",
+                                              "cpu_baseline", "batch", "layers", "steps",
+                                              "description") if k in o}
+            for o in others}
     return line
 
 
@@ -483,7 +638,8 @@ def run_e2e(r: Runner, stream, steps, device, world):
     Double-buffered as a serving loop would be: step i's inputs go up on one
     copy stream and step i-1's outputs come back on another while step i-1
     (then i) computes, each buffer set reused only after its previous step's
-    copies are done."""
+    copies are done.  The same loop runs untimed first (warm copy streams,
+    pinned buffers and graphs), then `steps` steps are timed."""
     w = r.w
     sets = [r, r.twin(stream)]
     hq = r.q.cpu().pin_memory()
@@ -497,45 +653,53 @@ def run_e2e(r: Runner, stream, steps, device, world):
     ev_in = [torch.cuda.Event() for _ in sets]     # inputs of the set's step are up
     ev_done = [torch.cuda.Event() for _ in sets]   # the set's step has computed
     ev_out = [torch.cuda.Event() for _ in sets]    # the set's outputs are down
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def loop(n, t0=None, t1=None):
+        if t0 is not None:
+            t0.record(stream)
+        up.wait_stream(stream)
+        down.wait_stream(stream)
+        for i in range(n):
+            k = i % 2
+            R = sets[k]
+            v = i % w.num_steps
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(ev_done[k])      # step i-2 has read this set's inputs
+                R.q.copy_(hq, non_blocking=True)
+                R.k.copy_(hk, non_blocking=True)
+                R.v.copy_(hv, non_blocking=True)
+                R.seq_lens[v].copy_(hsl[v], non_blocking=True)
+                ev_in[k].record(up)
+            stream.wait_event(ev_in[k])
+            if i >= 2:
+                stream.wait_event(ev_out[k])       # step i-2's outputs have left this set
+            with torch.cuda.stream(stream):
+                R.replay(i)
+                ev_done[k].record(stream)
+            down.wait_event(ev_done[k])
+            with torch.cuda.stream(down):
+                hout[k].copy_(R.out, non_blocking=True)
+                ev_out[k].record(down)
+        for k in range(min(n, len(sets))):
+            stream.wait_event(ev_out[k])
+        if t1 is not None:
+            t1.record(stream)
+        stream.synchronize()
+
+    loop(max(4, min(steps, 20)))   # warm: streams, pinned buffers, the twin's graphs
+    t0, t1 = _events()
     barrier()
     torch.cuda.synchronize()
-    t0.record(stream)
-    up.wait_event(t0)
-    down.wait_event(t0)
-    for i in range(steps):
-        k = i % 2
-        R = sets[k]
-        v = i % w.num_steps
-        with torch.cuda.stream(up):
-            if i >= 2:
-                up.wait_event(ev_done[k])      # step i-2 has read this set's inputs
-            R.q.copy_(hq, non_blocking=True)
-            R.k.copy_(hk, non_blocking=True)
-            R.v.copy_(hv, non_blocking=True)
-            R.seq_lens[v].copy_(hsl[v], non_blocking=True)
-            ev_in[k].record(up)
-        stream.wait_event(ev_in[k])
-        if i >= 2:
-            stream.wait_event(ev_out[k])       # step i-2's outputs have left this set
-        with torch.cuda.stream(stream):
-            R.replay(i)
-            ev_done[k].record(stream)
-        down.wait_event(ev_done[k])
-        with torch.cuda.stream(down):
-            hout[k].copy_(R.out, non_blocking=True)
-            ev_out[k].record(down)
-    for k in range(len(sets)):
-        stream.wait_event(ev_out[k])
-    t1.record(stream)
-    stream.synchronize()
+    loop(steps, t0, t1)
     barrier()
     ms = max_over_ranks(t0.elapsed_time(t1), device)
     return {"value": whole_job_rate(steps * w.num_layers * w.batch * r.queries, world, ms),
             "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps,
             "overlap": "double-buffered: host-to-device copies, step graphs and device-to-host "
-                       "copies on three streams"}
+                       "copies on three streams; the loop runs untimed first, then %d timed "
+                       "steps" % steps}
 
 
 def run_fill(r: Runner, stream, steps, device):
@@ -575,7 +739,7 @@ def run_fill(r: Runner, stream, steps, device):
         launch()
     for _ in range(3):
         g.replay()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0, t1 = _events()
     barrier()
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
@@ -588,6 +752,7 @@ def run_fill(r: Runner, stream, steps, device):
     ms = max_over_ranks(t0.elapsed_time(t1), device)
     if pkv.get_device_error(r.pool, stream) != 0:
         raise RuntimeError("device error in pkv_fill")
+    del g
     launches = steps * w.num_layers
     avg_s = ms / launches / 1e3
     peak, peak_kind = measured_peaks()
@@ -603,15 +768,16 @@ def run_fill(r: Runner, stream, steps, device):
 # ------------------------------------------------------------ oracle arms --
 
 def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None, max_layers=None,
-                  threads=None):
-    """Time the FP64 oracle on whole-layer append + decode of step 1 (all
-    sequences of the batch), cycling over `layers`, until `max_seconds` of
-    oracle time have passed (at least one layer; at most `max_layers`).
-    Each layer's pages are copied to the host once; repeats append the same
-    token again, which rewrites the same bits.  Returns (queries, seconds,
-    threads, layer-decodes done)."""
+                  threads=None, rows=None):
+    """Time the FP64 oracle on whole-layer append + decode of step 1 (the
+    sequences `rows`, all by default), cycling over `layers`, until
+    `max_seconds` of oracle time have passed (at least one layer; at most
+    `max_layers`).  Each layer's pages are copied to the host once; repeats
+    append the same token again, which rewrites the same bits.  Returns
+    (queries, seconds, threads, layer-decodes done)."""
     import oracle
     layers = list(range(w.num_layers)) if layers is None else list(layers)
+    rows = list(range(w.batch)) if rows is None else list(rows)
     threads = threads or os.cpu_count() or 1
     sl = w.seq_lens(1)
     cache = {}
@@ -619,18 +785,22 @@ def oracle_sample(w: W.Workload, pool_t, max_seconds: float, layers=None, max_la
     while True:
         l = layers[done % len(layers)]
         if l not in cache:
-            pool_h, bt_h = W.compact_pages(w, pool_t, range(w.batch), [l])
+            pool_h, bt_h = W.compact_pages(w, pool_t, rows, [l])
             q, k, v = W.step_inputs(w, 1, l, pool_t.device)
-            cache[l] = (pool_h, bt_h, W.bits(q), W.bits(k), W.bits(v))
-        pool_h, bt_h, qb, kb, vb = cache[l]
+            # sequences outside `rows` have no pages in the compact pool: give
+            # them length 0 (skipped by append and decode)
+            sl_rows = np.zeros_like(sl)
+            sl_rows[rows] = sl[rows]
+            cache[l] = (pool_h, bt_h, W.bits(q), W.bits(k), W.bits(v), sl_rows)
+        pool_h, bt_h, qb, kb, vb, sl_rows = cache[l]
         t = time.perf_counter()
-        oracle.append(pool_h, bt_h, sl, kb, vb, l)
-        oracle.decode(qb, pool_h, bt_h, sl, l, w.scale, nthreads=threads)
+        oracle.append(pool_h, bt_h[:, rows], sl_rows[rows], kb[rows], vb[rows], l)
+        oracle.decode(qb, pool_h, bt_h, sl_rows, l, w.scale, rows=rows, nthreads=threads)
         secs += time.perf_counter() - t
         done += 1
         if secs >= max_seconds or (max_layers is not None and done >= max_layers):
             break
-    return done * w.batch, secs, threads, done
+    return done * len(rows), secs, threads, done
 
 
 def cpu_model() -> str:
@@ -645,17 +815,23 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(w, pool_t, max_seconds):
-    q, s, thr, layers = oracle_sample(w, pool_t, max_seconds, max_layers=4096)
-    q1, s1, _, layers1 = oracle_sample(w, pool_t, max_seconds / 4, max_layers=4096, threads=1)
+def cpu_baseline(w, pool_t, max_seconds, rows=None):
+    """The FP64 oracle on the host cores (all threads, then one) on whole
+    layers of step 1 (`rows`: a sample of the batch, reported as such)."""
+    q, s, thr, layers = oracle_sample(w, pool_t, max_seconds, max_layers=4096, rows=rows)
+    q1, s1, _, layers1 = oracle_sample(w, pool_t, max_seconds / 4, max_layers=4096, threads=1,
+                                       rows=rows)
+    nrows = w.batch if rows is None else len(rows)
+    what = "whole-layer" if rows is None else \
+        "%d-of-%d-sequence (extrapolated: the rate per sequence is the same)" % (nrows, w.batch)
     return {"value": q / s, "unit": UNIT, "cores": thr, "kind": "oracle",
-            "sample": "%d whole-layer append+decode(s) of step 1, cycling over the %d layers "
+            "sample": "%d %s append+decode(s) of step 1, cycling over the %d layers "
                       "(%d sequences each), %.1f s of FP64 oracle work" %
-                      (layers, w.num_layers, w.batch, s),
+                      (layers, what, w.num_layers, nrows, s),
             "cpu_model": cpu_model(),
             "single_core_value": q1 / s1,
-            "single_core_sample": "%d whole-layer append+decode(s) on 1 thread, %.1f s" %
-                                  (layers1, s1)}
+            "single_core_sample": "%d %s append+decode(s) on 1 thread, %.1f s" %
+                                  (layers1, what, s1)}
 
 
 def run_reference(args, rank, world, local_rank):
@@ -720,6 +896,59 @@ def run_reference(args, rank, world, local_rank):
     }
 
 
+# ------------------------------------------------------------------ table --
+
+# Workloads whose layer fits in L2 (26.9 MB and 0.1 MB of K/V): reported hot
+# and cold.
+COLD_WORKLOADS = ("tiny", "llama1b_b16")
+# Sampled CPU baseline for the 35 GB workload (8 of its 256 sequences).
+STRESS_CPU_ROWS = [0, 37, 64, 101, 128, 199, 230, 255]
+
+
+def run_table(args, rank, world, local_rank):
+    """Every workload and option row of the measured-results table in one
+    run, on the current kernel sources: JSON line per row, then markdown."""
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    rows = []
+
+    def add(label, name, **kw):
+        rec = measure(args, name, device, rank, world, local_rank, **kw)
+        if rec is not None:
+            rec["row"] = label
+            print(json.dumps(rec), flush=True)
+            rows.append(rec)
+
+    for name in ("tiny", "llama1b_b16", "continuous_batching_b64", "long_context_b4",
+                 "stress_b256"):
+        add(name, name, full=name != "stress_b256", cold=name in COLD_WORKLOADS,
+            cpu_seconds=0.0 if args.no_cpu_baseline else 3.0,
+            cpu_rows=STRESS_CPU_ROWS if name == "stress_b256" else None)
+    for name, qs in (("continuous_batching_b64", (2, 4, 8)), ("long_context_b4", (2, 8))):
+        for q in qs:
+            add("%s, %d queries" % (name, q), name, queries=q)
+    add("continuous_batching_b64, BF16 output", "continuous_batching_b64", out_dtype="bf16")
+    if rank != 0:
+        return
+    print("| row | us per launch | alg. GB/s | of peak | cold L2: us, of peak | "
+          "decode-queries/s (step) | e2e | fill GB/s (of peak) | CPU oracle (cores) | "
+          "SM MHz (samples, reasons) |")
+    print("|---|---|---|---|---|---|---|---|---|---|")
+    for r in rows:
+        rf, c = r["roofline"], r["clocks"]
+        cold = r.get("cold_l2")
+        e2e = r.get("e2e")
+        fill = r.get("prefill_fill")
+        cpu = r.get("cpu_baseline")
+        print("| %s | %.2f | %.0f | %.1f %% | %s | %.4g | %s | %s | %s | %s (%d, %s) |" % (
+            r["row"], rf["avg_launch_us"], rf["achieved"], 100 * rf["frac"],
+            "%.2f, %.1f %%" % (cold["us_per_launch"], 100 * cold["frac"]) if cold else "-",
+            r["value"], "%.4g" % e2e["value"] if e2e else "-",
+            "%.0f (%.1f %%)" % (fill["achieved"], 100 * fill["frac"]) if fill else "-",
+            "%.4g (%d)" % (cpu["value"], cpu["cores"]) if cpu else "-",
+            c.get("sm_mhz"), c.get("samples", 0), ",".join(c.get("reasons", [])) or "none"))
+
+
 # --------------------------------------------------------------------- main --
 
 def main():
@@ -730,14 +959,23 @@ def main():
     ap.add_argument("--workload", default="continuous_batching_b64", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "mma"])
-    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--clock-seconds", type=float, default=1.0,
+                    help="replay the step graphs at least this long with the clock sampler on")
+    ap.add_argument("--also", default=None,
+                    help="comma-separated workloads measured beside the main one (default: "
+                         "long_context_b4,llama1b_b16 for the default workload; 'none')")
+    ap.add_argument("--cold-l2", action="store_true",
+                    help="also time the main workload with L2 flushed before every step")
+    ap.add_argument("--table", action="store_true",
+                    help="measure every workload and option row; print JSON lines and a table")
     ap.add_argument("--reference-seconds", type=float, default=60.0,
                     help="oracle time the --impl reference run spends in its timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fill", action="store_true", help="skip the prefill fill timing")
     ap.add_argument("--no-early-pages", action="store_true",
-                    help="wait for the preceding kernel before the first page loads")
+                    help="wait for the preceding kernels before the first page loads")
     ap.add_argument("--queries", type=int, default=1, choices=range(1, 9),
                     help="queries per sequence (> 1: causal among them, decode only)")
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])
@@ -750,6 +988,14 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.also is None:
+        args.also = ["long_context_b4", "llama1b_b16"] \
+            if args.workload == "continuous_batching_b64" else []
+    else:
+        args.also = [] if args.also in ("", "none") else args.also.split(",")
+    for name in args.also:
+        if name not in W.WORKLOADS:
+            ap.error("unknown workload %s" % name)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -762,6 +1008,9 @@ def main():
     try:
         if args.impl == "reference":
             line = run_reference(args, rank, world, local_rank)
+        elif args.table:
+            run_table(args, rank, world, local_rank)
+            line = None
         else:
             line = run_ours(args, rank, world, local_rank)
         if line is not None and rank == 0:
