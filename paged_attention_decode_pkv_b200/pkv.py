@@ -8,8 +8,11 @@ libpkv.so is missing or cannot be loaded, importing this module raises.
 """
 from __future__ import annotations
 
+import atexit
 import ctypes
 import os
+import sys
+import weakref
 from typing import Optional
 
 import torch
@@ -155,12 +158,32 @@ def _dev(t: torch.Tensor, dtype, shape, name):
     return ctypes.c_void_p(t.data_ptr())
 
 
+# Pools still open.  They are closed by an exit hook that runs before the
+# interpreter starts tearing modules down (and before torch's and the CUDA
+# runtime's own shutdown), while the device, the library and every object
+# the pool refers to are still alive; a pool that is only garbage-collected
+# during interpreter shutdown makes no CUDA call at all (its device memory
+# goes with the process).
+_LIVE_POOLS = weakref.WeakSet()
+
+
+@atexit.register
+def _close_live_pools():
+    for p in list(_LIVE_POOLS):
+        try:
+            p.close()
+        except Exception:
+            pass
+
+
 class Pool:
     """A pool of 32 KiB pages ([K|V][8 kv heads][16 slots][64] BF16 each).
 
     The page storage is a torch tensor owned by this object
     (``self.storage``, bfloat16 [num_pages, 2, 8, 16, 64]) or one the caller
-    passes in; the C library only borrows it.
+    passes in; the C library only borrows it.  CUDA graphs that captured
+    calls on a pool hold the addresses of its storage and workspaces:
+    release them before those tensors are freed.
     """
 
     def __init__(self, num_pages: int, storage: Optional[torch.Tensor] = None, device=None):
@@ -179,6 +202,7 @@ class Pool:
                                        storage.numel() * 2, ctypes.byref(self._h)),
                    "pkv_pool_create")
         self._ws = {}
+        _LIVE_POOLS.add(self)
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -192,13 +216,19 @@ class Pool:
             ws.zero_()
 
     def close(self):
+        """Destroy the C pool (synchronises its device).  Idempotent."""
         if self._h:
             with torch.cuda.device(self.device):
                 lib.pkv_pool_destroy(self._h)
             self._h = ctypes.c_void_p()
         self._ws.clear()
+        _LIVE_POOLS.discard(self)
 
     def __del__(self):
+        # During interpreter shutdown the CUDA runtime, torch's CUDA state or
+        # this module's globals may already be gone: make no device call then.
+        if sys.is_finalizing():
+            return
         try:
             self.close()
         except Exception:
