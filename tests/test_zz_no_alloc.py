@@ -69,3 +69,17 @@ def test_noalloc_rejects_batches_beyond_the_scratch():
         pkv.decode_noalloc(q, g.pool, bt, sl, 0, 0.125, out)
     assert e.value.status == pkv.ERR_TOO_LARGE
     assert "scratch" in pkv.lib.pkv_last_error_message().decode()
+
+
+def test_noalloc_long_batch_then_short_batch():
+    # A long-context call leaves many more split records in the shared scratch
+    # than the next, shorter call writes; the shorter call must read only its
+    # own (checked against the workspace entry point and the oracle).
+    long_ = GpuCase(make_case([6000, 4100, 2500], seed=606, spare_pages=2))
+    short = GpuCase(make_case([700, 30, 1500, 5, 260], seed=707, spare_pages=2))
+    assert max_err(_noalloc(long_), long_.oracle()) <= ATOL
+    for g in (short, long_, short):
+        got = _noalloc(g)
+        assert max_err(got, g.decode()) <= ATOL
+        assert max_err(got, g.oracle()) <= ATOL
+    assert pkv.get_device_error(short.pool) == 0
