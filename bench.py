@@ -379,10 +379,9 @@ class Runner:
         return tot / n
 
     def kernels_per_layer(self, decode_only=False):
-        """Kernels one layer of a step launches: the decode kernel (its
-        split-KV merge runs inside it), plus the separate append unless
-        fused."""
-        return 1 + (0 if self.fused or decode_only or self.queries > 1 else 1)
+        """Kernels one layer of a step launches: the decode kernel and the
+        split-KV merge, plus the separate append unless fused."""
+        return 2 + (0 if self.fused or decode_only or self.queries > 1 else 1)
 
     def close(self):
         """Release the graphs (they hold this library's kernel nodes), the
@@ -536,17 +535,17 @@ def measure(args, name, device, rank, world, local_rank, *, full=False, cold=Fal
             "frac": achieved / peak, "traffic": recorded_traffic(w.name, avg_bytes)
             if r.queries == 1 and out_dtype == "f32" else None,
             "peak_kind": peak_kind,
-            "kernel": "decode_kernel%s (split-KV merge inside)" %
+            "kernel": "decode_kernel%s (+ split-KV merge_kernel)" %
                       (" with fused append" if fused else ""),
             "alg_bytes_per_launch": avg_bytes, "avg_launch_us": avg_dec_s * 1e6,
             "launches": dec_launches},
         "gpu_launches": args.steps * layers * r.kernels_per_layer() +
                         (0 if fused else dec_launches * r.kernels_per_layer(decode_only=True)),
-        "decode_timing": ("CUDA events around the %d full-step replays (one fused append + "
-                          "decode launch per layer, %d launches)" % (args.steps, dec_launches)
+        "decode_timing": ("CUDA events around the %d full-step replays (fused append + decode "
+                          "+ merge per layer, %d launches)" % (args.steps, dec_launches)
                           if fused else
                           "CUDA events around %d back-to-back replays of the step's decode "
-                          "calls alone (one decode launch per layer, %d launches)" %
+                          "calls alone (decode + merge per layer, %d launches)" %
                           (args.steps, dec_launches)),
         "clocks": clocks,
         "kernel_source_sha256": kernel_source_digest(),
@@ -562,7 +561,7 @@ def measure(args, name, device, rank, world, local_rank, *, full=False, cold=Fal
         rec["append"] = {
             "kernel": "append_kernel", "us_per_launch": append_us,
             "bytes_per_launch": w.batch * (2 * 2048 + 8),
-            "how": "unfused step time minus decode time, per layer (PDL-chained)"}
+            "how": "unfused step time minus decode + merge time, per layer (PDL-chained)"}
     if e2e is not None:
         rec["e2e"] = e2e
     if fill is not None:
@@ -598,7 +597,7 @@ def run_ours(args, rank, world, local_rank):
             "kv_bytes_per_layer": m["kv_bytes_per_layer"], "accumulate": "f32",
             "kernel": m["kernel"], "parallelism": "dp%d (independent replicas)" % world,
             "queries_per_sequence": m["queries_per_sequence"], "out_dtype": m["out_dtype"],
-            "launch": "one CUDA graph per step (16 x %s)%s" %
+            "launch": "one CUDA graph per step (16 x %s + split merge)%s" %
                       ("fused append+decode" if m["fused"] else
                        "%d-query decode" % m["queries_per_sequence"]
                        if m["queries_per_sequence"] > 1 else "append + decode",

@@ -144,9 +144,8 @@ PKV_API int32_t pkv_pool_num_pages(const pkv_pool *pool);
  * before the preceding kernels of the stream have finished, so its set-up
  * overlaps them.  Every kernel of this library lets the next launch start
  * early, so "preceding kernels" means every earlier kernel of the stream
- * that may still be running, not only the one launched just before (a
- * decode's last CTAs can still run while the next decode starts, for
- * instance).
+ * that may still be running, not only the one launched just before (the
+ * previous decode can still run beside its split-KV merge, for instance).
  * The caller guarantees that none of them writes seq_lens or the block
  * tables (an append or a decode, which only read them, is fine).
  * PKV_LAUNCH_EARLY_PAGES (only together with both) lets decode also start
@@ -254,19 +253,12 @@ PKV_API int pkv_allocator_free(pkv_page_allocator *alloc, const int32_t *pages, 
 
 /*
  * Workspace bytes paged_attention_decode needs for this batch on the pool's
- * device.  The workspace is caller-owned device memory, 256-byte aligned,
- * laid out as
- *  - PKV_WORKSPACE_COUNTER_BYTES (512 KiB) of split-KV arrival counters:
- *    they must be zero before the workspace's first use (zero-fill the
- *    whole workspace once, e.g. cudaMemsetAsync), and every call leaves them
- *    at zero again -- also a call that reports a device error -- so a
- *    workspace can be reused for any batch without clearing;
- *  - then the partial results of split sequences (m, l and the unnormalised
- *    output of every piece: (batch + grid) * 8 * 1056 bytes per query, grid
- *    being the decode CTAs), which need no initialisation.
- * Calls that share one workspace must not overlap in time.
+ * device: the split-KV partial results (m, l and the unnormalised output of
+ * every piece of a split sequence).  The workspace is caller-owned device
+ * memory, 256-byte aligned; its contents need no initialisation (every
+ * decode writes what it later reads).  Calls that share one workspace must
+ * not overlap in time.
  */
-#define PKV_WORKSPACE_COUNTER_BYTES (512u << 10)
 PKV_API int pkv_decode_workspace_bytes(const pkv_pool *pool, int32_t batch, size_t *bytes_out);
 
 /*
@@ -274,16 +266,13 @@ PKV_API int pkv_decode_workspace_bytes(const pkv_pool *pool, int32_t batch, size
  *   out[b][h][:] = sum_{t<L} softmax_t(scale * q[b][h].K[t][h/4]) V[t][h/4]
  * with K/V read in place from the pages block_tables[layer][b][*], FP32
  * online softmax and FP32 accumulation.  Sequences with L == 0 get an
- * all-zero output.  One kernel launch: long contexts are split across the
- * GPU (split-KV), each CTA holding a piece writes its partial result to the
- * workspace, and the CTA that completes a sequence's pieces merges them
- * with log-sum-exp weights, in piece order (in groups of 8 pieces first for
- * sequences split further), so results do not depend on timing or on which
- * CTA merges; no CTA ever waits for another.  Device errors:
+ * all-zero output.  Long contexts are split across the GPU (split-KV): the
+ * decode kernel writes the pieces to the workspace and a second kernel,
+ * launched right after it on the same stream, merges them with log-sum-exp
+ * weights in a fixed order (results do not depend on timing).  Device errors:
  * L < 0 or L > max_blocks*16 -> PKV_ERR_BAD_SEQ_LEN (that row is written as
  * zeros); a page outside the pool -> PKV_ERR_BAD_PAGE (that page is
- * skipped).  Requires 8 * batch * max_blocks < 2^31 and batch + grid <=
- * 65536 (else PKV_ERR_UNSUPPORTED).  Every CTA keeps the
+ * skipped).  Requires 8 * batch * max_blocks < 2^31.  Every CTA keeps the
  * batch's lengths and page-count prefix in shared memory (8 bytes per
  * sequence): above about 4,000 sequences the tensor-core kernel runs one
  * CTA per SM instead of two, and above about 18,000 the call returns
@@ -433,17 +422,15 @@ PKV_API int pkv_gather(const pkv_pool *pool, const int32_t *block_tables, const 
  *  - Limit: returns PKV_ERR_TOO_LARGE (nothing launched) when the batch
  *    needs more scratch than that, i.e. when pkv_decode_workspace_bytes for
  *    this pool and batch (the exact check) exceeds it.  That size is
- *    PKV_WORKSPACE_COUNTER_BYTES + (batch + grid) * 8 * 1056 bytes, grid
- *    being the decode kernel's CTAs (SM count x CTAs per SM: 296 on a B200
- *    while the batch is small enough for two CTAs per SM), so a B200 takes
- *    up to 1,627 sequences.
+ *    (batch + grid) * 8 * 1056 bytes, grid being the decode kernel's CTAs
+ *    (SM count x CTAs per SM: 296 on a B200 while the batch is small enough
+ *    for two CTAs per SM), so a B200 takes up to 1,689 sequences.
  *  - Every call looks up the scratch's device address (cudaGetSymbolAddress,
  *    with the pool's device current; nothing is allocated).  The first
  *    lookup on a device may load the library's device code: make the first
  *    call before any stream capture.
  *  - All calls on one device share the one scratch area, which keeps the
- *    last call's contents (it starts zeroed, and every call leaves its
- *    counter area at zero, so no call has to clear it).  Calls whose
+ *    last call's contents; nothing in it has to start at zero.  Calls whose
  *    kernels overlap on the GPU (different streams, or different threads
  *    without ordering) race on it and give wrong results: serialise them.
  */

@@ -650,23 +650,24 @@ __device__ __forceinline__ OutRowsT<kBf16> out_rows(const DecodeArgs& a, int b, 
 //   M[h] = max_s m_s[h],  w_s[h] = exp2(m_s[h] - M[h]),
 //   S[h] = sum_s w_s[h] l_s[h],  O[h][d] = sum_s w_s[h] acc_s[h][d].
 // With `final_out`, query final_q's rows of it get O / S (zero where S == 0);
-// otherwise (M, S, O) is written as one partial record at `out` (which may
-// be P[0] itself: every lane reads the parts of P[0] it later writes before
-// writing anything).  Pieces are taken 32 at a time (running max rescaled
-// between groups, a fixed order): lane s reads m and l of piece s, and every
-// lane accumulates dims 2*lane, 2*lane+1 of the 4 heads with the loads of
-// kMergeBatch pieces in flight.  Records are read from L2 (ld.global.cg):
-// other CTAs wrote them.
+// otherwise (M, S, O) is written as one partial record at `out`.  Pieces are taken 32 at a time
+// (running max rescaled between groups, a fixed order): lane s reads m and l
+// of piece s, and every lane accumulates dims 2*lane, 2*lane+1 of the 4 heads
+// with the loads of kMergeBatch pieces in flight (4: the merge kernel's
+// register cap leaves no room for 8 without spilling).  kShared: P lives in
+// shared memory (plain loads) instead of global memory (L2 loads).
 constexpr int kMergeBatch = 4;
 
-__device__ __forceinline__ float4 ldcg4(const float* p) {
-  return __ldcg(reinterpret_cast<const float4*>(p));
+template <bool kShared>
+__device__ __forceinline__ float4 ld4(const float* p) {
+  return kShared ? *reinterpret_cast<const float4*>(p) : __ldcg(reinterpret_cast<const float4*>(p));
 }
-__device__ __forceinline__ float2 ldcg2(const float* p) {
-  return __ldcg(reinterpret_cast<const float2*>(p));
+template <bool kShared>
+__device__ __forceinline__ float2 ld2(const float* p) {
+  return kShared ? *reinterpret_cast<const float2*>(p) : __ldcg(reinterpret_cast<const float2*>(p));
 }
 
-template <class Out>
+template <bool kShared, class Out>
 __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stride, float* out,
                                                const Out* final_out, int final_q, int lane) {
   const bool final = final_out != nullptr;
@@ -688,13 +689,13 @@ __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stri
     for (int kk = 0; kk < kMergeBatch; ++kk)
 #pragma unroll
       for (int h = 0; h < kGroup; ++h)
-        v[kk][h] = (kk < n) ? ldcg2(base + kk * step + h * kDim + 2 * lane)
+        v[kk][h] = (kk < n) ? ld2<kShared>(base + kk * step + h * kDim + 2 * lane)
                             : make_float2(0.f, 0.f);
     float mm[kGroup] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     float ll[kGroup] = {0.f, 0.f, 0.f, 0.f};
     if (lane < n) {
       const float* p = P + (s0 + lane) * step;
-      const float4 m4 = ldcg4(p), l4 = ldcg4(p + 4);
+      const float4 m4 = ld4<kShared>(p), l4 = ld4<kShared>(p + 4);
       mm[0] = m4.x; mm[1] = m4.y; mm[2] = m4.z; mm[3] = m4.w;
       ll[0] = l4.x; ll[1] = l4.y; ll[2] = l4.z; ll[3] = l4.w;
     }
@@ -722,7 +723,7 @@ __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stri
         for (int kk = 0; kk < kMergeBatch; ++kk)
 #pragma unroll
           for (int h = 0; h < kGroup; ++h)
-            v[kk][h] = (k0 + kk < n) ? ldcg2(base + (k0 + kk) * step + h * kDim + 2 * lane)
+            v[kk][h] = (k0 + kk < n) ? ld2<kShared>(base + (k0 + kk) * step + h * kDim + 2 * lane)
                                      : make_float2(0.f, 0.f);
       }
 #pragma unroll
@@ -757,12 +758,11 @@ __device__ __forceinline__ void merge_partials(const float* P, int cnt, int stri
 }
 
 // Split-KV bookkeeping of sequence b: the CTA range of its first page and
-// its number of pieces K (CTAs its pages span).  Piece i of the sequence is
-// the one CTA c_first + i holds.  Partial records live at [g][b + cta], so
-// the pieces of one (sequence, kv head) unit are the consecutive slots
-// S0 .. S0 + K - 1 with S0 = g * (B + grid) + b + c_first (b + cta is
-// distinct for every piece of head g because both only grow along the page
-// order).
+// its number of pieces (CTAs its pages span).  Partial records live at
+// [g][b + cta], so the pieces of one (sequence, kv head) unit are the
+// consecutive slots S0 .. S0 + K - 1 with S0 = g * (B + grid) + b + c_first
+// (b + cta is distinct for every piece of head g because both only grow
+// along the page order).
 __device__ __forceinline__ int2 split_of(int64_t pages_before, int b, int np, int64_t chunk) {
   if (np == 0) return make_int2(0, 0);
   const int64_t first = pages_before + static_cast<int64_t>(kSeqCost) * b + kSeqCost;
@@ -780,42 +780,13 @@ __device__ __forceinline__ int64_t range_chunk(int64_t total_pages, int batch, i
   return chunk < 1 ? 1 : chunk;
 }
 
-// Split pieces of the CTA range holding pages [p0, p1): at most two, the
-// range's first sequence (if it began in an earlier range) and its last one
-// (if it continues in a later range) -- every other sequence of the range
-// lies wholly inside it; one if the range lies inside one sequence.
-struct Pending {
-  int n;       // 0, 1 or 2
-  int b0, b1;  // their sequences, in range order
-};
-
-__device__ __forceinline__ Pending range_pieces(const int32_t* s_pfx, int B, int32_t p0,
-                                                int32_t p1) {
-  Pending pend;
-  pend.n = 0;
-  pend.b0 = pend.b1 = 0;
-  if (p1 <= p0) return pend;
-  int bf, bl, j;
-  locate(s_pfx, B, p0, bf, j);
-  locate(s_pfx, B, p1 - 1, bl, j);
-  if (s_pfx[bf] < p0 || s_pfx[bf + 1] > p1) {
-    pend.b0 = bf;
-    pend.n = 1;
-  }
-  if (bl != bf && (s_pfx[bl] < p0 || s_pfx[bl + 1] > p1)) {
-    if (pend.n == 0) pend.b0 = bl; else pend.b1 = bl;
-    ++pend.n;
-  }
-  return pend;
-}
-
 // End of a sequence's piece inside this CTA's range, for kv head g (= this
 // warp): finish it in registers when the CTA holds the whole sequence, else
-// store the piece's partial record, counted in at the end of the range
-// (merge_split_units).
+// store the piece for the merge kernel that follows.
 template <class C>
-__device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a, int b, int g,
-                                           int j0, int j1, int np, int lane) {
+__device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a,
+                                           const int32_t* s_pfx, int b, int g, int j0, int j1,
+                                           int np, int64_t chunk, int lane) {
   if (j0 == 0 && j1 == np - 1) {
     if (a.out_bf16)
       cmp.finalize(out_rows<true>(a, b, g), lane);
@@ -825,102 +796,6 @@ __device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a, in
   }
   const int64_t slot = static_cast<int64_t>(g) * (a.batch + gridDim.x) + b + blockIdx.x;
   cmp.store_partial(a.partials + slot * a.num_queries * kPartialFloats, a.num_queries, lane);
-}
-
-// ---------------------------------------------------------------------------
-// Split-KV merge, inside the decode kernel: whoever completes a unit merges
-// it, so no CTA waits for another and no second kernel is launched.
-//
-// Pieces are counted in at the end of their CTA's range (every range ends at
-// about the same time, so this delays nothing, and it keeps counter round
-// trips out of the page pipeline).  A sequence split into K <= kMergeGroup
-// pieces has one counter: the CTA whose piece makes it K merges the K
-// records into the output rows.  Longer ones are merged in two levels, so
-// that no single SM reads more than about kMergeGroup records per kv head:
-// pieces form groups of kMergeGroup consecutive pieces, each with a counter;
-// the CTA completing a group merges its records into the record of the
-// group's first piece (in place), then counts the group in on the
-// sequence's counter, and the CTA completing the last group merges the group
-// records into the output rows.  Merging is in piece order, so the result
-// does not depend on which CTA does it.  Counters go back to zero when their
-// unit or group is done, so every launch finds and leaves them at zero.
-// Warp g merges kv head g, each query of the sequence in turn.
-//
-// Memory ordering: every thread fences (gpu scope) after writing its
-// records, then the CTA synchronises before its counter increment; the
-// CTA that observes the final count fences before reading the records
-// through L2.
-// ---------------------------------------------------------------------------
-constexpr int kMergeGroup = 8;
-
-// Warp g: merge `cnt` records of kv head g, slots s0, s0 + st, ..., into the
-// record at slot s0 (to_out false) or into sequence b's output rows.
-__device__ __forceinline__ void merge_head(const DecodeArgs& a, int b, int64_t s0, int cnt,
-                                           int st, bool to_out, int g, int lane) {
-  const int nq = a.num_queries;
-  const int64_t head = static_cast<int64_t>(g) * (a.batch + gridDim.x);
-  for (int qi = 0; qi < nq; ++qi) {
-    float* P = a.partials + ((head + s0) * nq + qi) * kPartialFloats;
-    if (!to_out) {
-      merge_partials(P, cnt, st * nq, P, static_cast<const OutRowsT<false>*>(nullptr), 0, lane);
-    } else if (a.out_bf16) {
-      const OutRowsT<true> out = out_rows<true>(a, b, g);
-      merge_partials(P, cnt, st * nq, nullptr, &out, qi, lane);
-    } else {
-      const OutRowsT<false> out = out_rows<false>(a, b, g);
-      merge_partials(P, cnt, st * nq, nullptr, &out, qi, lane);
-    }
-  }
-}
-
-// Count one split piece of sequence b (held by this CTA) in, and merge what
-// it completes.  Called by every thread of the CTA (all arguments uniform).
-// s_arr: one int of shared memory.
-__device__ __forceinline__ void count_in_piece(const DecodeArgs& a, const int32_t* s_pfx,
-                                               int64_t chunk, int b, int32_t* s_arr) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t* unit_ctr = a.counters + b;
-  const int2 sp = split_of(s_pfx[b], b, s_pfx[b + 1] - s_pfx[b], chunk);
-  const int K = sp.y, c_first = sp.x;
-  const int j = (static_cast<int>(blockIdx.x) - c_first) / kMergeGroup;
-  const bool two = K > kMergeGroup;
-  // group counters: by the slot (< batch + grid) of the group's first piece
-  int32_t* ctr = two ? a.counters + kCounterSlots + b + c_first + kMergeGroup * j : unit_ctr;
-  const int need = two ? min(kMergeGroup, K - kMergeGroup * j) : K;
-  __syncthreads();   // s_arr is free; every thread's records are fenced
-  if (threadIdx.x == 0) s_arr[0] = atomicAdd(ctr, 1);
-  __syncthreads();
-  if (s_arr[0] != need - 1) return;   // another piece is still to come
-  __threadfence();
-  if (!two) {
-    merge_head(a, b, b + c_first, K, 1, true, warp, lane);
-    if (threadIdx.x == 0) *ctr = 0;
-    return;
-  }
-  merge_head(a, b, b + c_first + kMergeGroup * j, need, 1, false, warp, lane);
-  __threadfence();   // the group record, before the count below
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    *ctr = 0;
-    s_arr[0] = atomicAdd(unit_ctr, 1);
-  }
-  __syncthreads();
-  if (s_arr[0] != (K + kMergeGroup - 1) / kMergeGroup - 1) return;
-  __threadfence();
-  merge_head(a, b, b + c_first, (K + kMergeGroup - 1) / kMergeGroup, kMergeGroup, true, warp,
-             lane);
-  if (threadIdx.x == 0) *unit_ctr = 0;
-}
-
-// Count this CTA's pieces in and merge the units or groups it completes, at
-// the end of its range (also after an aborted range: the counts must stay
-// exact whatever the records hold).
-__device__ __forceinline__ void merge_split_units(const DecodeArgs& a, const int32_t* s_pfx,
-                                                  int64_t chunk, const Pending& pend,
-                                                  int32_t* s_arr) {
-  __threadfence();   // this thread's records, before the counts
-  count_in_piece(a, s_pfx, chunk, pend.b0, s_arr);
-  if (pend.n > 1) count_in_piece(a, s_pfx, chunk, pend.b1, s_arr);
 }
 
 // Producer-side description of page f (this lane's slot of a 32-page batch):
@@ -1150,7 +1025,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
         if (lane == 0) record_error(a.err, kErrTimeout);
         s_flags[kS] = 1;
         drain(r);
-        break;
+        return;
       }
       issue(rr + kS, kIssuePage | kIssueRows);
     }
@@ -1160,11 +1035,11 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
       if (lane == 0) record_error(a.err, kErrTimeout);
       s_flags[kS] = 1;
       drain(r + 1);
-      break;
+      return;
     }
     if (s_flags[kS]) {   // another warp gave up; results are void
       drain(r + 1);
-      break;
+      return;
     }
     const uint32_t stage = base + L::stages + st * L::kStageBytes;
     if (need_q) {
@@ -1199,7 +1074,7 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + 8 * st);
     if (j == np - 1 || r == n - 1) {
-      flush_unit(cmp, a, b, warp, j_first, j, np, lane);
+      flush_unit(cmp, a, s_pfx, b, warp, j_first, j, np, chunk, lane);
       if (r < n - 1) {
         do {
           ++b;
@@ -1214,11 +1089,6 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
       ++j;
     }
   }
-  // Count this range's split pieces in (also after a timed-out wait, so
-  // that the counters stay exact) and merge the units this CTA completes.
-  const Pending pend = range_pieces(s_pfx, B, p0, p1);
-  if (pend.n > 0)
-    merge_split_units(a, s_pfx, chunk, pend, reinterpret_cast<int32_t*>(smem + L::tot));
 }
 
 template <class C>
@@ -1227,16 +1097,93 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
   decode_body<C>(tmap, a);
 }
 
-// The one-query tensor-core variant runs two CTAs per SM (shared memory
-// allows no third); its register cap only has to leave room for two.
-#ifndef PKV_Q1_MAX_REGS
-#define PKV_Q1_MAX_REGS 128
-#endif
-constexpr int kQ1Regs = PKV_Q1_MAX_REGS;
+// The one-query tensor-core variant needs no more than 88 registers per
+// thread without spilling.  Capped there, its two CTAs per SM leave 20,480
+// of the SM's 65,536 registers free: room for one merge CTA (256 threads at
+// the merge kernel's 80) beside them.  A merge CTA waiting for its decode
+// grid then no longer keeps the next layer's decode CTAs off its SM, so
+// that decode's first page loads (PKV_LAUNCH_EARLY_PAGES) overlap the merge.
+constexpr int kQ1Regs = 88;
 
 __global__ void __maxnreg__(kQ1Regs)
     decode_kernel_q1(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   decode_body<MmaComputeT<1, true>>(tmap, a);
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV merge: one CTA per (kv head g, sequence b) unit that decode split
+// into K > 1 pieces.  The split is recomputed here from the lengths (an
+// input that nothing in the launch writes), before waiting for the decode
+// grid, so that with programmatic dependent launch only the partial records
+// are read after decode ends.  Warp w merges pieces w, w + 8, ... into a
+// record in shared memory; warp 0 then merges the 8 records (a fixed order)
+// and writes the output rows.
+// ---------------------------------------------------------------------------
+constexpr int kMergeWarps = 8;
+
+// Three CTAs' worth of registers per SM (at most 85 per thread, 80 used):
+// one merge CTA fits beside two one-query decode CTAs (see decode_kernel_q1).
+template <int kNq, bool kBf16>   // kNq: queries per sequence, 0 = read from the arguments
+__global__ void __launch_bounds__(kMergeWarps * 32, 3)
+    merge_kernel(const DecodeArgs a, int32_t decode_grid) {
+  __shared__ __align__(16) float s_part[kMergeWarps][kPartialFloats];
+  __shared__ int32_t s_sum[2][kMergeWarps];
+  pdl_trigger();
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t cap = static_cast<int64_t>(a.max_blocks) * kTokens;
+  int before = 0, all = 0;
+  for (int i = threadIdx.x; i < a.batch; i += blockDim.x) {
+    int L = a.seq_lens[i];
+    if (L < 0 || L > cap || (L > 0 && L < a.num_queries)) L = 0;
+    const int np = (L + kTokens - 1) / kTokens;
+    all += np;
+    before += (i < b) ? np : 0;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    before += __shfl_xor_sync(kFull, before, off);
+    all += __shfl_xor_sync(kFull, all, off);
+  }
+  if (lane == 0) {
+    s_sum[0][warp] = before;
+    s_sum[1][warp] = all;
+  }
+  __syncthreads();
+  int64_t pages_before = 0, pages_all = 0;
+#pragma unroll
+  for (int k = 0; k < kMergeWarps; ++k) {
+    pages_before += s_sum[0][k];
+    pages_all += s_sum[1][k];
+  }
+  int Lb = a.seq_lens[b];
+  if (Lb < 0 || Lb > cap || (Lb > 0 && Lb < a.num_queries)) Lb = 0;
+  const int64_t chunk = range_chunk(pages_all, a.batch, decode_grid, a.min_chunk);
+  const int2 sp = split_of(pages_before, b, (Lb + kTokens - 1) / kTokens, chunk);
+  const int K = sp.y;
+  // This grid's completion is what the next programmatically dependent
+  // launch waits for, so it must imply decode's: CTA (0, 0) always waits for
+  // the decode grid; the other CTAs without work leave at once, freeing
+  // their SM slot for the next launch.
+  if (K <= 1 && (g | b) != 0) return;
+  pdl_wait();   // the pieces are written by the decode grid
+  if (K <= 1) return;
+  const int nq = kNq > 0 ? kNq : a.num_queries;   // kNq == 0: any count
+  const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + sp.x;
+  const int parts = min(kMergeWarps, K);
+  const OutRowsT<kBf16> out = out_rows<kBf16>(a, b, g);
+#pragma unroll
+  for (int qi = 0; qi < nq; ++qi) {   // a piece's record of query qi: slot * nq + qi
+    if (warp < parts) {
+      const int cnt = (K - warp + kMergeWarps - 1) / kMergeWarps;
+      merge_partials<false>(a.partials + ((S0 + warp) * nq + qi) * kPartialFloats, cnt,
+                            kMergeWarps * nq, s_part[warp],
+                            static_cast<const OutRowsT<kBf16>*>(nullptr), 0, lane);
+    }
+    __syncthreads();
+    if (warp == 0) merge_partials<true>(&s_part[0][0], parts, 1, nullptr, &out, qi, lane);
+    if (qi + 1 < nq) __syncthreads();   // s_part is rewritten for the next query
+  }
 }
 
 // ---------------------------------------------------------------- host side --
@@ -1333,11 +1280,8 @@ int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ct
   plan->threads = kWarps * 32;
   plan->smem = smem;
   plan->grid = grid_ctas > 0 ? grid_ctas : sm_count * per_sm;
-  if (static_cast<int64_t>(batch) + plan->grid > kCounterSlots) return PKV_ERR_UNSUPPORTED;
-  plan->counter_bytes = kCounterBytes;
   const int64_t slots = static_cast<int64_t>(kKvHeads) * (batch + plan->grid);
-  plan->ws_bytes = plan->counter_bytes +
-                   static_cast<size_t>(slots) * num_queries * kPartialFloats * sizeof(float);
+  plan->ws_bytes = static_cast<size_t>(slots) * num_queries * kPartialFloats * sizeof(float);
   return PKV_OK;
 }
 
@@ -1362,7 +1306,19 @@ cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const
   cudaError_t e = cudaErrorInvalidValue;
   with_compute(plan.kernel, plan.num_queries,
                [&](auto c) { e = launch_one<decltype(c)>(plan, tmap, a, flags, stream); });
-  return e;
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kKvHeads, a.batch);
+  cfg.blockDim = dim3(kMergeWarps * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
+  auto merge = a.num_queries == 1 ? (a.out_bf16 ? merge_kernel<1, true> : merge_kernel<1, false>)
+                                  : (a.out_bf16 ? merge_kernel<0, true> : merge_kernel<0, false>);
+  return cudaLaunchKernelEx(&cfg, merge, a, static_cast<int32_t>(plan.grid));
 }
 
 }  // namespace pkv

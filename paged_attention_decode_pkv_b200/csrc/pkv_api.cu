@@ -285,8 +285,7 @@ int decode_common(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_ne
   a.bt = layer_slab(block_tables, layer, batch, max_blocks);
   a.seq_lens = seq_lens;
   a.out = out;
-  a.counters = static_cast<int32_t*>(workspace);
-  a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + plan.counter_bytes);
+  a.partials = static_cast<float*>(workspace);
   a.err = pool->d_err;
   a.batch = batch;
   a.max_blocks = max_blocks;
@@ -465,9 +464,9 @@ int paged_attention_decode_noalloc(const uint16_t* q, const pkv_pool* pool,
   void* scratch = nullptr;
   s = scratch_address(&scratch);
   if (s != PKV_OK) return s;
-  // The scratch starts zeroed (static storage) and every decode leaves its
-  // counter area at zero again, so the shared scratch needs no clearing
-  // between calls.
+  // Nothing in the workspace has to start at zero (each decode writes the
+  // partial records before reading them), so the shared scratch needs no
+  // clearing between calls.
   return paged_attention_decode(q, pool, block_tables, seq_lens, layer, scale, out, num_layers,
                                 batch, max_blocks, scratch, sizeof(g_noalloc_scratch), stream);
 }

@@ -220,8 +220,6 @@ struct DecodeArgs {
   const int32_t* bt;        // this layer's block-table slab [B][max_blocks]
   const int32_t* seq_lens;  // [B]
   void* out;                // [B][num_queries][32][64], FP32 or BF16 (out_bf16)
-  int32_t* counters;        // split-KV arrival counters: [kCounterSlots] per sequence, then
-                            // [kCounterSlots] per group (by the slot of its first piece)
   float* partials;          // [8 kv heads][B + grid][num_queries][kPartialFloats]
   int32_t* err;             // sticky device error word
   int32_t batch;
@@ -246,19 +244,8 @@ struct DecodePlan {
   int grid;          // CTAs
   int threads;       // threads per CTA
   size_t smem;       // dynamic shared memory bytes
-  size_t counter_bytes;  // workspace bytes of the split-KV counters (at its start)
   size_t ws_bytes;   // workspace bytes
 };
-
-// Workspace layout: a fixed area of split-KV arrival counters (zero when no
-// launch runs), then the partial records.  The area's size and place do not
-// depend on the batch or the grid, so a workspace reused for another batch
-// never finds records where its counters are: kCounterSlots per-sequence
-// counters, then kCounterSlots per-group counters (indexed by a piece slot,
-// < batch + grid).
-constexpr int kCounterSlots = 1 << 16;
-constexpr size_t kCounterBytes = size_t(2) * kCounterSlots * sizeof(int32_t);   // 512 KiB
-static_assert(kCounterBytes == PKV_WORKSPACE_COUNTER_BYTES, "counter area of pkv.h");
 
 int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,
                 int num_queries, DecodePlan* plan);

@@ -47,7 +47,6 @@ ERR_BAD_SEQ_LEN = -8
 ERR_TOO_LARGE = -9
 ERR_APPEND_CONFLICT = -10
 NOALLOC_SCRATCH_BYTES = 16 << 20
-WORKSPACE_COUNTER_BYTES = 512 << 10
 
 EXPORTS = (
     "pkv_pool_create", "pkv_pool_destroy", "pkv_pool_data", "pkv_pool_num_pages", "pkv_append",
@@ -265,9 +264,7 @@ class Pool:
 
     def workspace(self, batch: int, kernel: int = KERNEL_AUTO, grid_ctas: int = 0,
                   num_queries: int = 1) -> torch.Tensor:
-        """A decode workspace, cached per (batch, kernel, grid, queries).
-        Zero-filled when made: its first WORKSPACE_COUNTER_BYTES are split-KV
-        counters that must start at zero (every call leaves them at zero)."""
+        """A decode workspace, cached per (batch, kernel, grid, queries)."""
         key = (int(batch), int(kernel), int(grid_ctas), int(num_queries))
         ws = self._ws.get(key)
         if ws is None:

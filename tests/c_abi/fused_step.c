@@ -82,7 +82,6 @@ int main(void) {
   CHECK(cudaMalloc((void**)&d_v, sizeof vn));
   CHECK(cudaMalloc((void**)&d_out, sizeof(float) * B * 32 * 64));
   CHECK(cudaMalloc(&d_ws, ws));
-  CHECK(cudaMemset(d_ws, 0, ws)); /* the split-KV counters start at zero */
   CHECK(cudaMemcpy(d_bt, bt, sizeof bt, cudaMemcpyHostToDevice));
   CHECK(cudaMemcpy(d_len, lens, sizeof lens, cudaMemcpyHostToDevice));
   CHECK(cudaMemcpy(d_q, q, sizeof q, cudaMemcpyHostToDevice));

@@ -154,7 +154,7 @@ def test_stress_batch256_sampled():
 
 # ---------------------------------------------------------------------------
 # The benchmarked launch itself: bench.py's Runner (one CUDA graph per step of
-# 16 fused append + decode calls), with bench.py's launch
+# 16 fused append + decode calls plus their merges), with bench.py's launch
 # flags (programmatic dependent launch, tables and first pages read before
 # the preceding kernels end), replayed step after step as the benchmark
 # replays it.  The only difference from the benchmark: before each step's

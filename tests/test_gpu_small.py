@@ -192,18 +192,14 @@ def test_programmatic_dependent_launch_keeps_results(kernel):
 @pytest.mark.parametrize("kernel", KERNELS)
 def test_bounded_wait_reports_timeout_and_context_survives(kernel):
     # A stage that nothing fills: every wait on it gives up after ~1 s, the
-    # kernel reports PKV_ERR_DEVICE_TIMEOUT, and the next launch works --
-    # on the same workspace, whose split-KV counters the aborted launch left
-    # at zero (its CTAs still count their pieces in).
+    # kernel reports PKV_ERR_DEVICE_TIMEOUT, and the next launch works.
     c = make_case([40, 300, 17], seed=37, spare_pages=2)
     g = GpuCase(c)
-    ws = g.pool.workspace(3, kernel)
     g.pool.set_launch_flags(pkv.LAUNCH_TEST_STALL)
-    g.decode(kernel=kernel, grid_ctas=7, workspace=ws)
+    g.decode(kernel=kernel)
     assert pkv.get_device_error(g.pool) == pkv.ERR_DEVICE_TIMEOUT
-    assert not ws[:pkv.WORKSPACE_COUNTER_BYTES].any()
     g.pool.set_launch_flags(0)
-    got = g.decode(kernel=kernel, grid_ctas=7, workspace=ws)
+    got = g.decode(kernel=kernel)
     assert pkv.get_device_error(g.pool) == 0
     assert max_err(got, g.oracle()) <= ATOL
 
@@ -212,41 +208,20 @@ def test_bounded_wait_reports_timeout_and_context_survives(kernel):
 @pytest.mark.parametrize("grid,min_chunk", [(0, 0), (7, 0), (0, 3), (400, 0), (600, 1)])
 def test_stale_workspace_contents_do_not_matter(kernel, grid, min_chunk):
     # The merge may only read partial records that this launch wrote: a
-    # workspace whose record area is full of earlier records (here: NaN
-    # bytes, and then the records of a different batch) must give the same
-    # result.  Its counter area must be zero, and every call leaves it so.
+    # workspace full of earlier records (here: NaN bytes, and then the
+    # records of a different batch) must give the same result.
     c = make_case([300, 1, 47, 129, 16, 517, 2], seed=41, spare_pages=5)
     g = GpuCase(c)
     want = g.oracle(scale=0.11)
     ws = g.pool.workspace(7, kernel, grid)
-    C = pkv.WORKSPACE_COUNTER_BYTES
-    ws[C:].fill_(0xFF)                   # every float of the records is NaN
+    ws.fill_(0xFF)                       # every float of it is NaN
     got = g.decode(scale=0.11, kernel=kernel, grid_ctas=grid, min_chunk=min_chunk, workspace=ws)
     assert np.isfinite(got).all()
     assert max_err(got, want) <= ATOL
-    assert not ws[:C].any()
     other = GpuCase(make_case([900, 33, 400, 5, 260, 1, 1200], seed=42, spare_pages=2))
     other.decode(kernel=kernel, grid_ctas=grid, min_chunk=min_chunk, workspace=ws)
-    assert not ws[:C].any()
     again = g.decode(scale=0.11, kernel=kernel, grid_ctas=grid, min_chunk=min_chunk, workspace=ws)
     assert np.array_equal(again, got)
-
-
-@pytest.mark.parametrize("kernel", KERNELS)
-def test_one_workspace_for_every_batch(kernel):
-    # One workspace sized for the largest batch serves smaller and larger
-    # batches in any order: records of a call never sit where a later call
-    # keeps its counters, and every call leaves the counters at zero.
-    small = GpuCase(make_case([40, 3000, 7], seed=51, spare_pages=2))
-    big = GpuCase(make_case([int(x) for x in np.random.default_rng(52).integers(1, 900, 300)],
-                            seed=53, spare_pages=2))
-    ws = torch.zeros(big.pool.workspace_bytes(300, kernel), dtype=torch.uint8, device="cuda")
-    C = pkv.WORKSPACE_COUNTER_BYTES
-    for g in (big, small, big, small):
-        got = g.decode(kernel=kernel, workspace=ws)
-        assert max_err(got, g.oracle()) <= ATOL
-        assert not ws[:C].any()
-        assert pkv.get_device_error(g.pool) == 0
 
 
 @pytest.mark.parametrize("batch", [3000, 5000])
