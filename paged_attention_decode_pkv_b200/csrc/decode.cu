@@ -838,16 +838,6 @@ struct SmemPlan {
   }
 };
 
-// Pages per CTA (counting the staged ones) whose loads may start before the
-// dependency wait with PKV_LAUNCH_EARLY_PAGES: the first kStages into shared
-// memory, the rest as L2 prefetches.  A one-wave grid of 296 CTAs then has
-// at most 296 x 6 x 32 KiB = 58 MB in flight, under half of the 126 MB L2.
-#ifndef PKV_L2_PREFETCH_PAGES
-#define PKV_L2_PREFETCH_PAGES 6
-#endif
-constexpr int kL2PrefetchPages = PKV_L2_PREFETCH_PAGES;
-static_assert(kL2PrefetchPages <= 32, "prefetched pages come from the first table batch");
-
 template <class C>
 __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const DecodeArgs& a) {
   constexpr int kS = C::kStages;
@@ -970,23 +960,12 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
   // last 16 steps' tokens lie in those two pages).  early_mask: pages r < kS
   // whose page part went out early.
   uint32_t early_mask = 0;
-  if (warp == 0 && early_pages) {
+  if (warp == 0 && early_pages)
     for (int r = 0; r < n && r < kS; ++r)
       if (!(__shfl_sync(kFull, cur_info, r & 31) & kInfoRecent)) {
         issue(r, kIssuePage);
         early_mask |= 1u << r;
       }
-    // The next pages of the range (beyond the stages) stream into L2 now as
-    // well, one lane per page, so that HBM keeps busy while the preceding
-    // kernels finish; their TMA loads then hit L2.  Capped at
-    // kL2PrefetchPages per CTA so that a wave's prefetches stay well inside
-    // L2.
-    if (lane >= kS && lane < n && lane < kL2PrefetchPages &&
-        static_cast<uint32_t>(cur_phys) < static_cast<uint32_t>(a.num_pages))
-      prefetch_l2(reinterpret_cast<const uint8_t*>(a.pool) +
-                      static_cast<int64_t>(cur_phys) * kPageBytes,
-                  kPageBytes);
-  }
   if (early) pdl_wait();
 
   // empty (or invalid) sequences: zero output rows, once across the grid

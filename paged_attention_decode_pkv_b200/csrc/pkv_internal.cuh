@@ -121,16 +121,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned) of global
-// memory into L2: a hint with no destination in shared memory and no
-// completion to wait for.  L2 is where every SM's writes meet, so a line
-// prefetched before another kernel writes it is never read stale.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
-               "r"(bytes)
-               : "memory");
-}
-
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
