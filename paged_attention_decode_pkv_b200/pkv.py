@@ -224,10 +224,11 @@ class Pool:
         self._ws.clear()
         _LIVE_POOLS.discard(self)
 
-    def __del__(self):
+    def __del__(self, _finalizing=sys.is_finalizing):
         # During interpreter shutdown the CUDA runtime, torch's CUDA state or
-        # this module's globals may already be gone: make no device call then.
-        if sys.is_finalizing():
+        # this module's globals (sys included: hence the bound default) may
+        # already be gone: make no device call then.
+        if _finalizing():
             return
         try:
             self.close()
