@@ -269,7 +269,10 @@ PKV_API int pkv_decode_workspace_bytes(const pkv_pool *pool, int32_t batch, size
  * all-zero output.  Long contexts are split across the GPU (split-KV): the
  * decode kernel writes the pieces to the workspace and a second kernel,
  * launched right after it on the same stream, merges them with log-sum-exp
- * weights in a fixed order (results do not depend on timing).  Device errors:
+ * weights in a fixed order (results do not depend on timing); above 512
+ * sequences the decode kernel also leaves the merge one split-table entry
+ * per CTA, so the merge's set-up does not grow with the square of the
+ * batch.  Device errors:
  * L < 0 or L > max_blocks*16 -> PKV_ERR_BAD_SEQ_LEN (that row is written as
  * zeros); a page outside the pool -> PKV_ERR_BAD_PAGE (that page is
  * skipped).  Requires 8 * batch * max_blocks < 2^31.  Every CTA keeps the

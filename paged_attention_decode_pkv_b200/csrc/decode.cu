@@ -838,7 +838,10 @@ struct SmemPlan {
   }
 };
 
-template <class C>
+// kTable: the batch is above kMergeScanMaxBatch, so the merge kernel reads
+// its splits from a table this kernel writes (a separate instantiation, so
+// that smaller batches run exactly the code without it).
+template <class C, bool kTable>
 __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const DecodeArgs& a) {
   constexpr int kS = C::kStages;
   using L = SmemPlan<C>;
@@ -968,6 +971,21 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
       }
   if (early) pdl_wait();
 
+  // Large batches: publish the split sequence whose first piece this CTA
+  // holds -- the range's last sequence, if it starts in the range and
+  // continues past it -- for the merge kernel (after the wait: the previous
+  // merge on this workspace reads the table until then).
+  if (kTable && threadIdx.x == 0) {
+    int2 e = make_int2(-1, 0);
+    if (n > 0) {
+      int bl, jl;
+      locate(s_pfx, B, p1 - 1, bl, jl);
+      if (s_pfx[bl] >= p0 && s_pfx[bl + 1] > p1)
+        e = make_int2(bl, split_of(s_pfx[bl], bl, s_pfx[bl + 1] - s_pfx[bl], chunk).y);
+    }
+    a.split_table[blockIdx.x] = e;
+  }
+
   // empty (or invalid) sequences: zero output rows, once across the grid
   for (int b = blockIdx.x * kWarps + warp; b < B; b += G * kWarps)
     if (s_pfx[b + 1] == s_pfx[b]) zero_rows(a, b, lane);
@@ -1070,10 +1088,10 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
   }
 }
 
-template <class C>
+template <class C, bool kTable>
 __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
-  decode_body<C>(tmap, a);
+  decode_body<C, kTable>(tmap, a);
 }
 
 // The one-query tensor-core variant needs no more than 88 registers per
@@ -1084,9 +1102,10 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
 // that decode's first page loads (PKV_LAUNCH_EARLY_PAGES) overlap the merge.
 constexpr int kQ1Regs = 88;
 
+template <bool kTable>
 __global__ void __maxnreg__(kQ1Regs)
     decode_kernel_q1(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
-  decode_body<MmaComputeT<1, true>>(tmap, a);
+  decode_body<MmaComputeT<1, true>, kTable>(tmap, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -1102,53 +1121,72 @@ constexpr int kMergeWarps = 8;
 
 // Three CTAs' worth of registers per SM (at most 85 per thread, 80 used):
 // one merge CTA fits beside two one-query decode CTAs (see decode_kernel_q1).
-template <int kNq, bool kBf16>   // kNq: queries per sequence, 0 = read from the arguments
+// kNq: queries per sequence, 0 = read from the arguments; kTable: splits
+// from decode's table (batches above kMergeScanMaxBatch), else from the
+// lengths.
+template <int kNq, bool kBf16, bool kTable>
 __global__ void __launch_bounds__(kMergeWarps * 32, 3)
     merge_kernel(const DecodeArgs a, int32_t decode_grid) {
   __shared__ __align__(16) float s_part[kMergeWarps][kPartialFloats];
   __shared__ int32_t s_sum[2][kMergeWarps];
   pdl_trigger();
-  const int g = blockIdx.x, b = blockIdx.y;
+  const int g = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t cap = static_cast<int64_t>(a.max_blocks) * kTokens;
-  int before = 0, all = 0;
-  for (int i = threadIdx.x; i < a.batch; i += blockDim.x) {
-    int L = a.seq_lens[i];
-    if (L < 0 || L > cap || (L > 0 && L < a.num_queries)) L = 0;
-    const int np = (L + kTokens - 1) / kTokens;
-    all += np;
-    before += (i < b) ? np : 0;
-  }
+  int b, K, c_first;
+  if constexpr (!kTable) {
+    // CTA (g, b): sequence b's split, from the lengths
+    b = blockIdx.y;
+    const int64_t cap = static_cast<int64_t>(a.max_blocks) * kTokens;
+    int before = 0, all = 0;
+    for (int i = threadIdx.x; i < a.batch; i += blockDim.x) {
+      int L = a.seq_lens[i];
+      if (L < 0 || L > cap || (L > 0 && L < a.num_queries)) L = 0;
+      const int np = (L + kTokens - 1) / kTokens;
+      all += np;
+      before += (i < b) ? np : 0;
+    }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    before += __shfl_xor_sync(kFull, before, off);
-    all += __shfl_xor_sync(kFull, all, off);
-  }
-  if (lane == 0) {
-    s_sum[0][warp] = before;
-    s_sum[1][warp] = all;
-  }
-  __syncthreads();
-  int64_t pages_before = 0, pages_all = 0;
+    for (int off = 16; off > 0; off >>= 1) {
+      before += __shfl_xor_sync(kFull, before, off);
+      all += __shfl_xor_sync(kFull, all, off);
+    }
+    if (lane == 0) {
+      s_sum[0][warp] = before;
+      s_sum[1][warp] = all;
+    }
+    __syncthreads();
+    int64_t pages_before = 0, pages_all = 0;
 #pragma unroll
-  for (int k = 0; k < kMergeWarps; ++k) {
-    pages_before += s_sum[0][k];
-    pages_all += s_sum[1][k];
+    for (int k = 0; k < kMergeWarps; ++k) {
+      pages_before += s_sum[0][k];
+      pages_all += s_sum[1][k];
+    }
+    int Lb = a.seq_lens[b];
+    if (Lb < 0 || Lb > cap || (Lb > 0 && Lb < a.num_queries)) Lb = 0;
+    const int64_t chunk = range_chunk(pages_all, a.batch, decode_grid, a.min_chunk);
+    const int2 sp = split_of(pages_before, b, (Lb + kTokens - 1) / kTokens, chunk);
+    K = sp.y;
+    c_first = sp.x;
+    // This grid's completion is what the next programmatically dependent
+    // launch waits for, so it must imply decode's: CTA (0, 0) always waits
+    // for the decode grid; the other CTAs without work leave at once,
+    // freeing their SM slot for the next launch.
+    if (K <= 1 && (g | b) != 0) return;
+    pdl_wait();   // the pieces are written by the decode grid
+  } else {
+    // CTA (g, c): the split sequence whose first piece decode CTA c holds,
+    // from the table decode wrote (every CTA waits: the table comes from
+    // the decode grid)
+    pdl_wait();
+    c_first = blockIdx.y;
+    const int2 e = __ldcg(&a.split_table[c_first]);
+    b = e.x;
+    K = e.y;
+    if (b < 0) return;
   }
-  int Lb = a.seq_lens[b];
-  if (Lb < 0 || Lb > cap || (Lb > 0 && Lb < a.num_queries)) Lb = 0;
-  const int64_t chunk = range_chunk(pages_all, a.batch, decode_grid, a.min_chunk);
-  const int2 sp = split_of(pages_before, b, (Lb + kTokens - 1) / kTokens, chunk);
-  const int K = sp.y;
-  // This grid's completion is what the next programmatically dependent
-  // launch waits for, so it must imply decode's: CTA (0, 0) always waits for
-  // the decode grid; the other CTAs without work leave at once, freeing
-  // their SM slot for the next launch.
-  if (K <= 1 && (g | b) != 0) return;
-  pdl_wait();   // the pieces are written by the decode grid
   if (K <= 1) return;
   const int nq = kNq > 0 ? kNq : a.num_queries;   // kNq == 0: any count
-  const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + sp.x;
+  const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + c_first;
   const int parts = min(kMergeWarps, K);
   const OutRowsT<kBf16> out = out_rows<kBf16>(a, b, g);
 #pragma unroll
@@ -1168,17 +1206,17 @@ __global__ void __launch_bounds__(kMergeWarps * 32, 3)
 // ---------------------------------------------------------------- host side --
 
 // The kernel that runs compute type C.
-template <class C>
+template <class C, bool kTable>
 static auto decode_fn() {
   if constexpr (std::is_same_v<C, MmaComputeT<1, true>>)
-    return &decode_kernel_q1;
+    return &decode_kernel_q1<kTable>;
   else
-    return &decode_kernel<C>;
+    return &decode_kernel<C, kTable>;
 }
 
-template <class C>
+template <class C, bool kTable = false>
 static const void* kernel_ptr() {
-  return reinterpret_cast<const void*>(decode_fn<C>());
+  return reinterpret_cast<const void*>(decode_fn<C, kTable>());
 }
 
 // Tensor-core variants by queries per sequence: 1 (its own, fastest),
@@ -1207,9 +1245,11 @@ static bool with_compute(int kernel, int nq, F&& f) {
   return true;
 }
 
-static const void* kernel_for(int kernel, int nq) {
+static const void* kernel_for(int kernel, int nq, bool table = false) {
   const void* fn = nullptr;
-  with_compute(kernel, nq, [&](auto c) { fn = kernel_ptr<decltype(c)>(); });
+  with_compute(kernel, nq, [&](auto c) {
+    fn = table ? kernel_ptr<decltype(c), true>() : kernel_ptr<decltype(c), false>();
+  });
   return fn;
 }
 
@@ -1225,7 +1265,10 @@ cudaError_t prepare_decode_kernels(int device) {
   if (e != cudaSuccess) return e;
   for (const void* fn : {kernel_for(PKV_KERNEL_SIMT, 1), kernel_for(PKV_KERNEL_MMA, 1),
                           kernel_for(PKV_KERNEL_MMA, 2), kernel_for(PKV_KERNEL_MMA, 4),
-                          kernel_for(PKV_KERNEL_MMA, 6), kernel_for(PKV_KERNEL_MMA, 8)}) {
+                          kernel_for(PKV_KERNEL_MMA, 6), kernel_for(PKV_KERNEL_MMA, 8),
+                          kernel_for(PKV_KERNEL_SIMT, 1, true), kernel_for(PKV_KERNEL_MMA, 1, true),
+                          kernel_for(PKV_KERNEL_MMA, 2, true), kernel_for(PKV_KERNEL_MMA, 4, true),
+                          kernel_for(PKV_KERNEL_MMA, 6, true), kernel_for(PKV_KERNEL_MMA, 8, true)}) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, fn);
     if (e != cudaSuccess) return e;
@@ -1240,7 +1283,7 @@ int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ct
                 int num_queries, DecodePlan* plan) {
   if (num_queries < 1 || num_queries > kMaxQueries) return PKV_ERR_UNSUPPORTED;
   if (kernel == PKV_KERNEL_AUTO) kernel = PKV_KERNEL_MMA;
-  const void* fn = kernel_for(kernel, num_queries);
+  const void* fn = kernel_for(kernel, num_queries, batch > kMergeScanMaxBatch);
   if (!fn) return PKV_ERR_UNSUPPORTED;
   int optin = 0;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) !=
@@ -1260,7 +1303,8 @@ int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ct
   plan->smem = smem;
   plan->grid = grid_ctas > 0 ? grid_ctas : sm_count * per_sm;
   const int64_t slots = static_cast<int64_t>(kKvHeads) * (batch + plan->grid);
-  plan->ws_bytes = static_cast<size_t>(slots) * num_queries * kPartialFloats * sizeof(float);
+  plan->records_bytes = static_cast<size_t>(slots) * num_queries * kPartialFloats * sizeof(float);
+  plan->ws_bytes = plan->records_bytes + static_cast<size_t>(plan->grid) * sizeof(int2);
   return PKV_OK;
 }
 
@@ -1277,7 +1321,8 @@ static cudaError_t launch_one(const DecodePlan& plan, const CUtensorMap& tmap, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, decode_fn<C>(), tmap, a);
+  return a.batch > kMergeScanMaxBatch ? cudaLaunchKernelEx(&cfg, decode_fn<C, true>(), tmap, a)
+                                      : cudaLaunchKernelEx(&cfg, decode_fn<C, false>(), tmap, a);
 }
 
 cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const DecodeArgs& a,
@@ -1287,7 +1332,7 @@ cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const
                [&](auto c) { e = launch_one<decltype(c)>(plan, tmap, a, flags, stream); });
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kKvHeads, a.batch);
+  cfg.gridDim = dim3(kKvHeads, a.batch <= kMergeScanMaxBatch ? a.batch : plan.grid);
   cfg.blockDim = dim3(kMergeWarps * 32);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1295,8 +1340,14 @@ cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
-  auto merge = a.num_queries == 1 ? (a.out_bf16 ? merge_kernel<1, true> : merge_kernel<1, false>)
-                                  : (a.out_bf16 ? merge_kernel<0, true> : merge_kernel<0, false>);
+  const bool table = a.batch > kMergeScanMaxBatch;
+  auto merge =
+      table ? (a.num_queries == 1
+                   ? (a.out_bf16 ? merge_kernel<1, true, true> : merge_kernel<1, false, true>)
+                   : (a.out_bf16 ? merge_kernel<0, true, true> : merge_kernel<0, false, true>))
+            : (a.num_queries == 1
+                   ? (a.out_bf16 ? merge_kernel<1, true, false> : merge_kernel<1, false, false>)
+                   : (a.out_bf16 ? merge_kernel<0, true, false> : merge_kernel<0, false, false>));
   return cudaLaunchKernelEx(&cfg, merge, a, static_cast<int32_t>(plan.grid));
 }
 

@@ -286,6 +286,7 @@ int decode_common(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_ne
   a.seq_lens = seq_lens;
   a.out = out;
   a.partials = static_cast<float*>(workspace);
+  a.split_table = reinterpret_cast<int2*>(static_cast<uint8_t*>(workspace) + plan.records_bytes);
   a.err = pool->d_err;
   a.batch = batch;
   a.max_blocks = max_blocks;

@@ -211,6 +211,8 @@ struct DecodeArgs {
   const int32_t* seq_lens;  // [B]
   void* out;                // [B][num_queries][32][64], FP32 or BF16 (out_bf16)
   float* partials;          // [8 kv heads][B + grid][num_queries][kPartialFloats]
+  int2* split_table;        // [grid]: (sequence, pieces) of the split sequence whose first
+                            // piece each decode CTA holds, or (-1, 0); large batches only
   int32_t* err;             // sticky device error word
   int32_t batch;
   int32_t max_blocks;
@@ -227,6 +229,13 @@ struct DecodeArgs {
   __nv_bfloat16* pool;
 };
 
+// Batches up to this size: each merge CTA finds its split from the lengths
+// before its dependency wait (B loads, overlapping decode).  Larger ones:
+// decode publishes one split-table entry per CTA and the merge grid has one
+// CTA per (kv head, decode CTA), each reading its entry after the wait, so
+// the merge set-up no longer grows with the square of the batch.
+constexpr int kMergeScanMaxBatch = 512;
+
 // Launch planning shared by the workspace query and the launch.
 struct DecodePlan {
   int kernel;        // PKV_KERNEL_SIMT or PKV_KERNEL_MMA
@@ -234,7 +243,8 @@ struct DecodePlan {
   int grid;          // CTAs
   int threads;       // threads per CTA
   size_t smem;       // dynamic shared memory bytes
-  size_t ws_bytes;   // workspace bytes
+  size_t records_bytes;  // workspace bytes of the partial records (at its start)
+  size_t ws_bytes;   // workspace bytes: the records, then the split table [grid] int2
 };
 
 int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,

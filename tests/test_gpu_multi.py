@@ -164,3 +164,32 @@ def test_more_queries_than_context_is_reported():
     assert not got[0].any()
     want = oracle.decode_multi(q[1:], c["pool"], c["bt"][:, 1:], c["seq_lens"][1:], 0, 0.125)
     assert max_err(got[1:], want) <= ATOL
+
+
+@pytest.mark.parametrize("grid,nq,bf16", [(0, 1, False), (0, 2, True), (7, 1, False),
+                                          (400, 3, False), (50, 1, True)])
+def test_large_batch_split_table(grid, nq, bf16):
+    # Above 512 sequences the merge kernel takes each split from a table the
+    # decode CTAs write (one entry per CTA) instead of rescanning the
+    # lengths: long and short sequences mixed so that many are split, some
+    # over many CTAs, for one and several queries and both output types.
+    rng = np.random.default_rng(600 + grid + nq)
+    lens = [int(x) for x in rng.integers(nq, 400, 600)]
+    lens[5], lens[300], lens[599] = 3000, 0, 2500
+    c = make_case(lens, seed=601, spare_pages=2)
+    g = GpuCase(c)
+    q = _q2(c, 3, nq)
+    dt = torch.bfloat16 if bf16 else torch.float32
+    kw = dict(grid_ctas=grid, out_dtype=dt)
+    if nq == 1:
+        got = pkv.decode_general(u16_to_bf16(q[:, 0]), g.pool, g.bt, g.sl, 0, 0.125, **kw)
+        torch.cuda.synchronize()
+        got = _f64(got)[:, None]
+    else:
+        got = _f64(_run(g, q, nq, **kw))
+    assert pkv.get_device_error(g.pool) == 0
+    want = oracle.decode_multi(q, c["pool"], c["bt"], c["seq_lens"], 0, 0.125)
+    tol = ATOL + (2.0 ** -8 * np.abs(want).max() if bf16 else 0.0)
+    assert np.isfinite(got).all()
+    assert max_err(got, want) <= tol
+    assert not got[300].any()
