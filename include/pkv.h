@@ -425,9 +425,10 @@ PKV_API int pkv_gather(const pkv_pool *pool, const int32_t *block_tables, const 
  *  - Limit: returns PKV_ERR_TOO_LARGE (nothing launched) when the batch
  *    needs more scratch than that, i.e. when pkv_decode_workspace_bytes for
  *    this pool and batch (the exact check) exceeds it.  That size is
- *    (batch + grid) * 8 * 1056 bytes, grid being the decode kernel's CTAs
- *    (SM count x CTAs per SM: 296 on a B200 while the batch is small enough
- *    for two CTAs per SM), so a B200 takes up to 1,689 sequences.
+ *    (batch + grid) * 8 * 1056 + grid * 8 bytes, grid being the decode
+ *    kernel's CTAs (SM count x CTAs per SM: 296 on a B200 while the batch is
+ *    small enough for two CTAs per SM), so a B200 takes up to 1,689
+ *    sequences.
  *  - Every call looks up the scratch's device address (cudaGetSymbolAddress,
  *    with the pool's device current; nothing is allocated).  The first
  *    lookup on a device may load the library's device code: make the first
