@@ -263,13 +263,14 @@ class Runner:
     """Device-resident state of one workload on one GPU."""
 
     def __init__(self, w: W.Workload, device, kernel: int, fused: bool, queries: int = 1,
-                 out_dtype=torch.float32, grid: int = 0):
+                 out_dtype=torch.float32, grid: int = 0, min_chunk: int = 0):
         from paged_attention_decode_pkv_b200 import pkv
         self.pkv = pkv
         self.w = w
         self.device = device
         self.kernel = kernel
         self.grid = grid
+        self.min_chunk = min_chunk
         self.queries = queries
         self.out_dtype = out_dtype
         # two queries per sequence: decode only (their tokens would be
@@ -328,19 +329,20 @@ class Runner:
                 pkv.decode_general(self.q[l], self.pool, self.bt, sl, l, self.w.scale,
                                    num_queries=self.queries, out_dtype=self.out_dtype,
                                    out=self.out[l], workspace=self.ws, kernel=self.kernel,
-                                   grid_ctas=self.grid,
+                                   grid_ctas=self.grid, min_chunk=self.min_chunk,
                                    stream=stream, **kv)
                 continue
             if self.fused:
                 pkv.decode_append(self.q[l], self.k[l], self.v[l], self.pool, self.bt, sl, l,
                                   self.w.scale, out=self.out[l], workspace=self.ws,
-                                  kernel=self.kernel, grid_ctas=self.grid, stream=stream)
+                                  kernel=self.kernel, grid_ctas=self.grid,
+                                  min_chunk=self.min_chunk, stream=stream)
                 continue
             if not decode_only:
                 pkv.append(self.pool, self.bt, sl, self.k[l], self.v[l], l, stream=stream)
             pkv.decode(self.q[l], self.pool, self.bt, sl, l, self.w.scale, out=self.out[l],
                        workspace=self.ws, kernel=self.kernel, grid_ctas=self.grid,
-                       stream=stream)
+                       min_chunk=self.min_chunk, stream=stream)
 
     def capture(self, stream):
         """CUDA graphs, one per lengths variant (the workload's step cycle):
@@ -443,7 +445,7 @@ def measure(args, name, device, rank, world, local_rank, *, full=False, cold=Fal
     w = workload_for_rank(name, rank)
     fused = not args.unfused and queries == 1
     tdtype = torch.bfloat16 if out_dtype == "bf16" else torch.float32
-    r = Runner(w, device, kern, fused, queries, tdtype, args.grid)
+    r = Runner(w, device, kern, fused, queries, tdtype, args.grid, args.min_chunk)
     flags = launch_flags(pkv, pdl=not args.no_pdl, early_pages=not args.no_early_pages)
     r.pool.set_launch_flags(flags)
     stream = torch.cuda.Stream(device)
@@ -527,6 +529,7 @@ def measure(args, name, device, rank, world, local_rank, *, full=False, cold=Fal
         "workload": w.name, "description": w.description, "batch": w.batch, "layers": layers,
         "pool_pages": w.num_pages, "kv_bytes_per_layer": w.kv_bytes(1),
         "queries_per_sequence": r.queries, "out_dtype": out_dtype, "kernel": kname,
+        "grid": args.grid, "min_chunk": args.min_chunk,
         "fused": fused, "flags": flags, "steps": args.steps, "ms_per_step": ms / args.steps,
         "value": value, "unit": UNIT,
         "decode_queries_per_s": w.batch * r.queries / avg_dec_s,
@@ -981,6 +984,8 @@ def main():
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "bf16"])
     ap.add_argument("--grid", type=int, default=0,
                     help="decode CTAs (0: one persistent wave over the device)")
+    ap.add_argument("--min-chunk", type=int, default=0,
+                    help="minimum pages per decode CTA range (0: automatic)")
     ap.add_argument("--unfused", action="store_true",
                     help="separate append and decode launches instead of the fused call")
     ap.add_argument("--no-pdl", action="store_true",
