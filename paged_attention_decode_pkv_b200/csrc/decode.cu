@@ -1109,11 +1109,15 @@ __global__ void __maxnreg__(kQ1Regs)
 }
 
 // ---------------------------------------------------------------------------
-// Split-KV merge: one CTA per (kv head g, sequence b) unit that decode split
-// into K > 1 pieces.  The split is recomputed here from the lengths (an
-// input that nothing in the launch writes), before waiting for the decode
-// grid, so that with programmatic dependent launch only the partial records
-// are read after decode ends.  Warp w merges pieces w, w + 8, ... into a
+// Split-KV merge: one CTA per (kv head g, unit) for the (sequence, kv head)
+// units that decode split into K > 1 pieces.  Up to kMergeScanMaxBatch
+// sequences the grid is (8, batch) and each CTA recomputes its sequence's
+// split from the lengths (an input that nothing in the launch writes),
+// before waiting for the decode grid, so that with programmatic dependent
+// launch only the partial records are read after decode ends.  Above, the
+// grid is (8, decode CTAs) and CTA (g, c) reads, after the wait, the split
+// table entry decode CTA c wrote: the set-up no longer reads every length in
+// every one of 8 x batch CTAs.  Warp w merges pieces w, w + 8, ... into a
 // record in shared memory; warp 0 then merges the 8 records (a fixed order)
 // and writes the output rows.
 // ---------------------------------------------------------------------------
