@@ -175,3 +175,34 @@ def test_fused_rejects_missing_new_rows():
         g.q.data_ptr(), None, None, g.pool.handle, g.bt.data_ptr(), g.sl.data_ptr(), 0, 0.125,
         P.data_ptr(), 1, 2, g.bt.shape[2], ws.data_ptr(), ws.numel(), None)
     assert st == pkv.ERR_INVALID_ARG
+
+
+def test_large_batch_fused_chain_with_early_pages():
+    # Above 512 sequences decode writes the merge's split table right after
+    # its dependency wait, while the previous step's merge (which reads the
+    # table) may still be running beside the early part of this decode: a
+    # chain of fused steps with programmatic launch and early pages, every
+    # step checked against the oracle.
+    rng = np.random.default_rng(640)
+    lens0 = rng.integers(1, 300, 640).astype(np.int32)
+    lens0[[3, 333, 639]] = [2500, 1800, 3000]
+    steps = 4
+    c = make_case(list(lens0 + steps), seed=641, spare_pages=2)
+    g = GpuCase(c)
+    g.pool.set_launch_flags(EARLY_ALL)
+    host = c["pool"].copy()
+    from tests.cases import bf16_bits
+    outs, wants = [], []
+    for s in range(1, steps + 1):
+        sl = lens0 + s
+        k = bf16_bits(rng.standard_normal((640, 8, 64)))
+        v = bf16_bits(rng.standard_normal((640, 8, 64)))
+        outs.append(pkv.decode_append(g.q, u16_to_bf16(k), u16_to_bf16(v), g.pool, g.bt,
+                                      to_dev(sl), 0, 0.125))
+        oracle.append(host, c["bt"], sl, k, v, 0)
+        wants.append(oracle.decode(c["q"], host, c["bt"], sl, 0, 0.125))
+    torch.cuda.synchronize()
+    assert pkv.get_device_error(g.pool) == 0
+    assert np.array_equal(bits(g.pool_t).reshape(host.shape), host)
+    for s, (out, want) in enumerate(zip(outs, wants), 1):
+        assert max_err(out.cpu().numpy().astype(np.float64), want) <= ATOL, s
