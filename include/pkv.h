@@ -429,10 +429,12 @@ PKV_API int pkv_gather(const pkv_pool *pool, const int32_t *block_tables, const 
  *    kernel's CTAs (SM count x CTAs per SM: 296 on a B200 while the batch is
  *    small enough for two CTAs per SM), so a B200 takes up to 1,689
  *    sequences.
- *  - Every call looks up the scratch's device address (cudaGetSymbolAddress,
- *    with the pool's device current; nothing is allocated).  The first
- *    lookup on a device may load the library's device code: make the first
- *    call before any stream capture.
+ *  - The first call on a device looks up the scratch's device address
+ *    (cudaGetSymbolAddress, with the pool's device current; nothing is
+ *    allocated) and keeps it for the life of the process; make that first
+ *    call before any stream capture.  A reset of the device's context
+ *    (cudaDeviceReset, or the primary context torn down) invalidates the
+ *    kept address: do not call this entry point on that device afterwards.
  *  - All calls on one device share the one scratch area, which keeps the
  *    last call's contents; nothing in it has to start at zero.  Calls whose
  *    kernels overlap on the GPU (different streams, or different threads

@@ -3,6 +3,7 @@
 // Host-visible argument errors are caught here before anything is launched;
 // everything else is the kernels' business (see pkv.h for the contract).
 #include <cstdio>
+#include <mutex>
 #include <new>
 
 #include "append_check.cuh"
@@ -422,24 +423,30 @@ int pkv_get_device_error(pkv_pool* pool, pkv_stream_t stream, int32_t* status_ou
 // workspace.  The area is a file-scope __device__ array (so every GPU that
 // loads the library holds it until the process exits); its size bounds the
 // batch (pkv.h gives the limit).  The host needs the array's device address,
-// which is not the host-side symbol: it is looked up with
-// cudaGetSymbolAddress, with the pool's device current, on every call -- a
-// host-side lookup that allocates nothing and stays right after a device
-// reset, which would invalidate a cached address.  (The first lookup on a
-// device may load the library's device code, hence the rule in pkv.h that
-// the first call comes before any stream capture.)
+// which is not the host-side symbol: it is looked up once per device with
+// cudaGetSymbolAddress, with that device current, on the first call, and
+// kept for the life of the process (a reset of the device's context
+// invalidates it; pkv.h says so).
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-// Device address of the current device's scratch array.
-int scratch_address(void** out) {
-  void* p = nullptr;
-  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-  if (e != cudaSuccess || !p)
-    return from_cuda(e == cudaSuccess ? cudaErrorInvalidSymbol : e,
-                     "paged_attention_decode_noalloc: scratch address");
-  *out = p;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[256];   // per device ordinal; nullptr until looked up
+
+// Device address of this device's scratch array (looked up on first use,
+// with `device` current: the caller has checked that it is).
+int scratch_for_device(int device, void** out) {
+  if (device < 0 || device >= 256) return PKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[device]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return from_cuda(e == cudaSuccess ? cudaErrorInvalidSymbol : e,
+                                                 "paged_attention_decode_noalloc: scratch address");
+    g_scratch_addr[device] = p;
+  }
+  *out = g_scratch_addr[device];
   return PKV_OK;
 }
 }  // namespace
@@ -463,11 +470,11 @@ int paged_attention_decode_noalloc(const uint16_t* q, const pkv_pool* pool,
     return PKV_ERR_TOO_LARGE;
   }
   void* scratch = nullptr;
-  s = scratch_address(&scratch);
+  s = scratch_for_device(pool->device, &scratch);
   if (s != PKV_OK) return s;
   // Nothing in the workspace has to start at zero (each decode writes the
-  // partial records before reading them), so the shared scratch needs no
-  // clearing between calls.
+  // partial records and the split table before reading them), so the shared
+  // scratch needs no clearing between calls.
   return paged_attention_decode(q, pool, block_tables, seq_lens, layer, scale, out, num_layers,
                                 batch, max_blocks, scratch, sizeof(g_noalloc_scratch), stream);
 }
