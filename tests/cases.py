@@ -115,3 +115,45 @@ FILL_CONFLICT_CASES = [
     ("skipped sequence", [[4, 0], [4, 1]], [5, 5], [0, 30], False),
     ("empty sequences", [[2, 0], [2, 0], [2, 1]], [0, 0, 3], [0, 0, 0], False),
 ]
+
+
+def shared_prefix_case(seed=71, prefix_pages=3, tails=(5, 37, 16, 130, 1)):
+    """Sequences whose first prefix_pages pages are the same physical pages
+    (a common prompt prefix), each with its own tail pages; and the same
+    batch with the prefix copied into private pages."""
+    rng = np.random.default_rng(seed)
+    B = len(tails)
+    lens = np.array([16 * prefix_pages + t for t in tails], np.int32)
+    need = (lens + 15) // 16
+    own = need - prefix_pages
+    P_shared = prefix_pages + int(own.sum()) + 2
+    mb = int(need.max())
+    bt = np.full((1, B, mb), -1, np.int32)
+    perm = rng.permutation(P_shared).astype(np.int32)
+    bt[0, :, :prefix_pages] = perm[:prefix_pages]
+    cur = prefix_pages
+    for b in range(B):
+        bt[0, b, prefix_pages:need[b]] = perm[cur:cur + own[b]]
+        cur += own[b]
+    pool = np.full((P_shared, 2, 8, 16, 64), NAN, np.uint16)
+    for p in perm[:prefix_pages]:
+        pool[p] = bf16_bits(rng.standard_normal((2, 8, 16, 64)))
+    for b in range(B):
+        for t in range(16 * prefix_pages, int(lens[b])):
+            pool[bt[0, b, t // 16], :, :, t % 16, :] = bf16_bits(rng.standard_normal((2, 8, 64)))
+    q = bf16_bits(rng.standard_normal((B, 32, 64)))
+    k_new = np.stack([pool[bt[0, b, (lens[b] - 1) // 16], 0, :, (lens[b] - 1) % 16] for b in range(B)])
+    v_new = np.stack([pool[bt[0, b, (lens[b] - 1) // 16], 1, :, (lens[b] - 1) % 16] for b in range(B)])
+    shared = dict(pool=pool, bt=bt, seq_lens=lens, q=q, k_new=k_new, v_new=v_new)
+    # private copies of the prefix pages for every sequence but the first
+    extra = (B - 1) * prefix_pages
+    pool2 = np.concatenate([pool, np.full((extra, 2, 8, 16, 64), NAN, np.uint16)])
+    bt2 = bt.copy()
+    nxt = P_shared
+    for b in range(1, B):
+        for j in range(prefix_pages):
+            pool2[nxt] = pool[bt[0, b, j]]
+            bt2[0, b, j] = nxt
+            nxt += 1
+    private = dict(shared, pool=pool2, bt=bt2)
+    return shared, private

@@ -10,7 +10,7 @@ import torch
 import oracle
 from paged_attention_decode_pkv_b200 import pkv
 from paged_attention_decode_pkv_b200 import workloads as W
-from tests.cases import NAN, bf16_bits, make_case
+from tests.cases import NAN, bf16_bits, make_case, shared_prefix_case
 from tests.harness import ATOL, KERNELS, GpuCase, bits, max_err, to_dev, u16_to_bf16
 
 pytestmark = pytest.mark.gpu
@@ -243,3 +243,29 @@ def test_batch_beyond_shared_memory_is_unsupported():
     with pytest.raises(pkv.PkvError) as e:
         g.pool.workspace_bytes(20000)
     assert e.value.status == pkv.ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("fused", [False, True])
+def test_shared_prefix_pages_are_read_in_place(kernel, fused):
+    # several sequences read the same physical pages (a reused prefix,
+    # read-only): the result equals the oracle and, bit for bit, the same
+    # batch with the prefix in private pages; the fused call appends into
+    # each sequence's own last page only
+    shared, private = shared_prefix_case()
+    outs = []
+    for c in (shared, private):
+        g = GpuCase(c)
+        if fused:
+            got = pkv.decode_append(g.q, u16_to_bf16(c["k_new"]), u16_to_bf16(c["v_new"]), g.pool,
+                                    g.bt, g.sl, 0, 0.125, kernel=kernel)
+            torch.cuda.synchronize()
+            got = got.cpu().numpy().astype(np.float64)
+        else:
+            got = g.decode(kernel=kernel)
+        assert pkv.get_device_error(g.pool) == 0
+        assert max_err(got, g.oracle()) <= ATOL
+        if fused:   # only the appended slots were written, with the bits they held
+            assert np.array_equal(bits(g.pool_t).reshape(c["pool"].shape), c["pool"])
+        outs.append(got)
+    assert np.array_equal(outs[0], outs[1])

@@ -356,3 +356,18 @@ def test_decode_multi_rejects_a_query_without_tokens():
     with pytest.raises(oracle.OracleError):
         oracle.decode_multi(np.zeros((2, 2, H, D), np.uint16), c["pool"], c["bt"],
                             c["seq_lens"], 0, 0.125)
+
+
+def test_shared_pages_read_in_place_equal_private_copies():
+    # Pages that several sequences' tables name (a reused prompt prefix) are
+    # read in place ("Curso gratuito recorre la inferencia de LLM...",
+    # section on the KV cache: decode reads the pages where they are): the
+    # output is bitwise that of the same batch with the prefix copied into
+    # private pages.
+    from tests.cases import shared_prefix_case
+    shared, private = shared_prefix_case()
+    a = oracle.decode(shared["q"], shared["pool"], shared["bt"], shared["seq_lens"], 0, 0.125)
+    b = oracle.decode(private["q"], private["pool"], private["bt"], private["seq_lens"], 0, 0.125)
+    assert (shared["bt"][0, :, :3] == shared["bt"][0, 0, :3]).all()   # really shared
+    assert len(np.unique(private["bt"][0, :, :3])) == 3 * shared["bt"].shape[1]
+    assert np.array_equal(a, b)
