@@ -27,8 +27,9 @@ time, against the measured HBM copy bandwidth, with the DRAM traffic of the
 committed ncu capture.  ``clocks`` are sampled over the timed steps and a
 following window of at least --clock-seconds of the same graph replays
 (``clocks.window``: that window's own per-launch time).  ``per_workload``
-holds the same measurement for the other workloads the speed target names
-(long context, and the Llama-1B batch with a cold-L2 figure).  ``e2e`` is
+holds the same measurement for the other workloads (long context, the second
+speed target; the Llama-1B batch with a cold-L2 figure; the 35 GB stress
+batch).  ``e2e`` is
 the same step with its inputs and outputs crossing from and to pinned host
 memory every step; ``prefill_fill`` the page-fill bandwidth;
 ``cpu_baseline`` the FP64 oracle on the host cores.  ``--impl reference``
@@ -584,7 +585,8 @@ def run_ours(args, rank, world, local_rank):
     for name in args.also:
         rec = measure(args, name, device, rank, world, local_rank,
                       cold=name in COLD_WORKLOADS or args.cold_l2,
-                      cpu_seconds=0.0 if args.no_cpu_baseline else min(args.cpu_seconds, 3.0))
+                      cpu_seconds=0.0 if args.no_cpu_baseline else min(args.cpu_seconds, 3.0),
+                      cpu_rows=STRESS_CPU_ROWS if name == "stress_b256" else None)
         others.append(rec)
     if rank != 0:
         return None
@@ -968,7 +970,8 @@ def main():
                     help="replay the step graphs at least this long with the clock sampler on")
     ap.add_argument("--also", default=None,
                     help="comma-separated workloads measured beside the main one (default: "
-                         "long_context_b4,llama1b_b16 for the default workload; 'none')")
+                         "long_context_b4,llama1b_b16,stress_b256 for the default workload; "
+                         "'none')")
     ap.add_argument("--cold-l2", action="store_true",
                     help="also time the main workload with L2 flushed before every step")
     ap.add_argument("--table", action="store_true",
@@ -994,7 +997,7 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.also is None:
-        args.also = ["long_context_b4", "llama1b_b16"] \
+        args.also = ["long_context_b4", "llama1b_b16", "stress_b256"] \
             if args.workload == "continuous_batching_b64" else []
     else:
         args.also = [] if args.also in ("", "none") else args.also.split(",")
