@@ -109,3 +109,60 @@ def test_fifo_admission_loop_runs_every_request_within_the_pool():
     assert done == set(range(len(need))) - {17}
     assert order == sorted(order)     # admitted in arrival order
     assert a.free_count == P
+
+
+def test_random_operations_match_a_free_stack_model():
+    # Thousands of random allocs and frees (good and bad) against a plain
+    # Python model of the documented policy: a LIFO stack of free pages
+    # (page 0 on top when fresh), all-or-nothing allocation, TOO_LARGE above
+    # the pool size, OUT_OF_PAGES above the free count, and frees validated
+    # as a whole (in range, held, listed once) before any page goes back.
+    import random
+    from paged_attention_decode_pkv_b200 import pkv
+    rng = random.Random(2024)
+    for n in (1, 7, 64, 300):
+        a = pkv.PageAllocator(n)
+        stack = list(range(n - 1, -1, -1))   # top = end
+        held = set()
+        for _ in range(3000):
+            if rng.random() < 0.55:
+                count = rng.choice([0, 1, 2, rng.randint(0, n), n, n + 1])
+                if count > n:
+                    want = pkv.ERR_TOO_LARGE
+                elif count > len(stack):
+                    want = pkv.ERR_OUT_OF_PAGES
+                else:
+                    want = pkv.OK
+                if want == pkv.OK:
+                    got = a.alloc(count)
+                    exp = [stack.pop() for _ in range(count)]
+                    assert got == exp
+                    held.update(exp)
+                else:
+                    with pytest.raises(pkv.PkvError) as e:
+                        a.alloc(count)
+                    assert e.value.status == want
+            else:
+                pages = rng.sample(sorted(held), rng.randint(0, len(held))) if held else []
+                bad = rng.random() < 0.3
+                if bad:
+                    kind = rng.choice(["range", "free", "twice"])
+                    if kind == "range":
+                        pages = pages + [rng.choice([-1, n, n + 5])]
+                    elif kind == "free" and len(held) < n:
+                        pages = pages + [rng.choice(sorted(set(range(n)) - held))]
+                    elif kind == "twice" and pages:
+                        pages = pages + [pages[0]]
+                    else:
+                        bad = False
+                if bad:
+                    with pytest.raises(pkv.PkvError) as e:
+                        a.free(pages)
+                    assert e.value.status == pkv.ERR_INVALID_ARG
+                else:
+                    a.free(pages)
+                    stack.extend(pages)
+                    held.difference_update(pages)
+            assert a.free_count == len(stack)
+            assert len(stack) + len(held) == n
+        a.close()
