@@ -413,6 +413,20 @@ def _replays(r: Runner, stream, steps, decode_only=False, start=0):
     return e0, e1
 
 
+def _replays_each(r: Runner, stream, steps, start=0):
+    """`steps` back-to-back step replays with an event after each one (the
+    events sit between graph launches, never inside a graph).  Returns the
+    first and last events and the per-step durations (ms) after a sync."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    with torch.cuda.stream(stream):
+        evs[0].record(stream)
+        for i in range(steps):
+            r.replay(start + i)
+            evs[i + 1].record(stream)
+    stream.synchronize()
+    return evs[0], evs[-1], [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+
+
 def _cold_replays(r: Runner, stream, steps, decode_only=False):
     """Per-step CUDA-event times (ms) with L2 flushed before every step: a
     buffer twice the L2 size is written between replays, outside the
@@ -479,8 +493,7 @@ def measure(args, name, device, rank, world, local_rank, *, full=False, cold=Fal
         ms = t0.elapsed_time(t1)
         n_win = max(1, int(math.ceil(args.clock_seconds * 1e3 / max(ms / args.steps, 1e-3))))
         n_win = min(n_win, 2_000_000)
-        w0, w1 = _replays(r, stream, n_win, start=args.steps)
-        stream.synchronize()
+        w0, w1, per_step = _replays_each(r, stream, n_win, start=args.steps)
     barrier()
     torch.cuda.synchronize()
     layers = w.num_layers
@@ -525,6 +538,7 @@ def measure(args, name, device, rank, world, local_rank, *, full=False, cold=Fal
                 "step graphs right after them" % (args.steps, n_win),
         "seconds": (ms + win_ms) / 1e3, "replays": n_win,
         "us_per_launch": win_ms / (n_win * layers) * 1e3,
+        "median_us_per_launch": statistics.median(per_step) / layers * 1e3,
         "achieved_gbs": win_achieved, "frac": win_achieved / peak}
     rec = {
         "workload": w.name, "description": w.description, "batch": w.batch, "layers": layers,
