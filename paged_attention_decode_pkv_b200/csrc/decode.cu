@@ -645,116 +645,16 @@ __device__ __forceinline__ OutRowsT<kBf16> out_rows(const DecodeArgs& a, int b, 
   return OutRowsT<kBf16>{static_cast<T*>(a.out) + e, kQHeads * kDim};
 }
 
-// Fixed-order log-sum-exp merge of `cnt` partial records P[0], P[stride],
-// ... (pieces of one (sequence, kv head) unit, in piece order):
-//   M[h] = max_s m_s[h],  w_s[h] = exp2(m_s[h] - M[h]),
-//   S[h] = sum_s w_s[h] l_s[h],  O[h][d] = sum_s w_s[h] acc_s[h][d].
-// With `final_out`, query final_q's rows of it get O / S (zero where S == 0);
-// otherwise (M, S, O) is written as one partial record at `out`.  Pieces are taken 32 at a time
-// (running max rescaled between groups, a fixed order): lane s reads m and l
-// of piece s, and every lane accumulates dims 2*lane, 2*lane+1 of the 4 heads
-// with the loads of kMergeBatch pieces in flight (4: the merge kernel's
-// register cap leaves no room for 8 without spilling).  kShared: P lives in
-// shared memory (plain loads) instead of global memory (L2 loads).
-constexpr int kMergeBatch = 4;
-
-template <bool kShared>
-__device__ __forceinline__ float4 ld4(const float* p) {
-  return kShared ? *reinterpret_cast<const float4*>(p) : __ldcg(reinterpret_cast<const float4*>(p));
+// Split-KV merge staging: the merge kernel copies the records of a
+// (sequence, kv head) unit from the workspace into shared memory with
+// cp.async (L2 only: the records were written by the decode grid just
+// before), all of them in one round when they fit, so that the merge waits
+// for a single L2 round trip instead of one per batch of register loads.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-template <bool kShared>
-__device__ __forceinline__ float2 ld2(const float* p) {
-  return kShared ? *reinterpret_cast<const float2*>(p) : __ldcg(reinterpret_cast<const float2*>(p));
-}
-
-template <bool kShared, class Out>
-__device__ __forceinline__ void merge_partials(const float* P, int cnt, int stride, float* out,
-                                               const Out* final_out, int final_q, int lane) {
-  const bool final = final_out != nullptr;
-  const int64_t step = static_cast<int64_t>(stride) * kPartialFloats;
-  float M[kGroup], S[kGroup];
-  float2 O[kGroup];
-#pragma unroll
-  for (int h = 0; h < kGroup; ++h) {
-    M[h] = -INFINITY;
-    S[h] = 0.f;
-    O[h] = make_float2(0.f, 0.f);
-  }
-  for (int s0 = 0; s0 < cnt; s0 += 32) {
-    const int n = min(32, cnt - s0);
-    const float* base = P + s0 * step + 2 * kGroup;
-    // accumulator loads of the first kMergeBatch pieces go out with the m/l loads
-    float2 v[kMergeBatch][kGroup];
-#pragma unroll
-    for (int kk = 0; kk < kMergeBatch; ++kk)
-#pragma unroll
-      for (int h = 0; h < kGroup; ++h)
-        v[kk][h] = (kk < n) ? ld2<kShared>(base + kk * step + h * kDim + 2 * lane)
-                            : make_float2(0.f, 0.f);
-    float mm[kGroup] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    float ll[kGroup] = {0.f, 0.f, 0.f, 0.f};
-    if (lane < n) {
-      const float* p = P + (s0 + lane) * step;
-      const float4 m4 = ld4<kShared>(p), l4 = ld4<kShared>(p + 4);
-      mm[0] = m4.x; mm[1] = m4.y; mm[2] = m4.z; mm[3] = m4.w;
-      ll[0] = l4.x; ll[1] = l4.y; ll[2] = l4.z; ll[3] = l4.w;
-    }
-    float wgt[kGroup];
-#pragma unroll
-    for (int h = 0; h < kGroup; ++h) {
-      float mc = mm[h];
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) mc = fmaxf(mc, __shfl_xor_sync(kFull, mc, off));
-      const float mn = fmaxf(M[h], mc);
-      if (mn != -INFINITY) {   // rescale what was accumulated under the old max
-        const float r = fast_exp2(M[h] - mn);
-        S[h] *= r;
-        O[h].x *= r;
-        O[h].y *= r;
-      }
-      M[h] = mn;
-      // a piece whose pages were all skipped has m = -inf and weight 0
-      wgt[h] = (mm[h] == -INFINITY) ? 0.f : fast_exp2(mm[h] - mn);
-      S[h] = fmaf(wgt[h], ll[h], S[h]);
-    }
-    for (int k0 = 0; k0 < n; k0 += kMergeBatch) {
-      if (k0 > 0) {
-#pragma unroll
-        for (int kk = 0; kk < kMergeBatch; ++kk)
-#pragma unroll
-          for (int h = 0; h < kGroup; ++h)
-            v[kk][h] = (k0 + kk < n) ? ld2<kShared>(base + (k0 + kk) * step + h * kDim + 2 * lane)
-                                     : make_float2(0.f, 0.f);
-      }
-#pragma unroll
-      for (int kk = 0; kk < kMergeBatch; ++kk)
-#pragma unroll
-        for (int h = 0; h < kGroup; ++h) {
-          const float wk = __shfl_sync(kFull, wgt[h], (k0 + kk) & 31);
-          O[h].x = fmaf(wk, v[kk][h].x, O[h].x);
-          O[h].y = fmaf(wk, v[kk][h].y, O[h].y);
-        }
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < kGroup; ++h)
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) S[h] += __shfl_xor_sync(kFull, S[h], off);
-  if (final) {
-#pragma unroll
-    for (int h = 0; h < kGroup; ++h) {
-      const float inv = S[h] > 0.f ? 1.f / S[h] : 0.f;
-      final_out->put2(final_q, h, 2 * lane, O[h].x * inv, O[h].y * inv);
-    }
-  } else {
-    if (lane == 0) {
-      reinterpret_cast<float4*>(out)[0] = make_float4(M[0], M[1], M[2], M[3]);
-      reinterpret_cast<float4*>(out)[1] = make_float4(S[0], S[1], S[2], S[3]);
-    }
-#pragma unroll
-    for (int h = 0; h < kGroup; ++h)
-      reinterpret_cast<float2*>(out + 2 * kGroup + h * kDim)[lane] = O[h];
-  }
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // Split-KV bookkeeping of sequence b: the CTA range of its first page and
@@ -1097,7 +997,7 @@ __global__ void __launch_bounds__(kWarps * 32, C::kMinBlocks)
 // The one-query tensor-core variant needs no more than 88 registers per
 // thread without spilling.  Capped there, its two CTAs per SM leave 20,480
 // of the SM's 65,536 registers free: room for one merge CTA (256 threads at
-// the merge kernel's 80) beside them.  A merge CTA waiting for its decode
+// up to 80 registers) beside them.  A merge CTA waiting for its decode
 // grid then no longer keeps the next layer's decode CTAs off its SM, so
 // that decode's first page loads (PKV_LAUNCH_EARLY_PAGES) overlap the merge.
 constexpr int kQ1Regs = 88;
@@ -1117,22 +1017,40 @@ __global__ void __maxnreg__(kQ1Regs)
 // launch only the partial records are read after decode ends.  Above, the
 // grid is (8, decode CTAs) and CTA (g, c) reads, after the wait, the split
 // table entry decode CTA c wrote: the set-up no longer reads every length in
-// every one of 8 x batch CTAs.  Warp w merges pieces w, w + 8, ... into a
-// record in shared memory; warp 0 then merges the 8 records (a fixed order)
-// and writes the output rows.
+// every one of 8 x batch CTAs.
+//
+// The merge itself is the fixed-order log-sum-exp combination of the unit's
+// pieces s = 0 .. K-1 (in piece order), per head h of the group:
+//   M[h] = max_s m_s[h],  w_s[h] = exp2(m_s[h] - M[h]) (0 where m_s = -inf),
+//   S[h] = sum_s w_s[h] l_s[h],  out[h][d] = (sum_s w_s[h] acc_s[h][d]) / S[h]
+// (zero where S == 0).  The records are staged in shared memory `chunk` at a
+// time (one round for every unit of up to `chunk` pieces; a running max
+// rescales between rounds).  Per round, warp h < 4 computes head h's weights
+// (lane s holds pieces s and s + 32) and the round's share of S; then each of
+// the 256 threads accumulates one output element (h, d) over the round's
+// pieces in order.
 // ---------------------------------------------------------------------------
-constexpr int kMergeWarps = 8;
+constexpr int kMergeThreads = kGroup * kDim;   // one output element per thread
+constexpr int kMergeWarps = kMergeThreads / 32;
+constexpr int kMergeMaxChunk = 64;             // pieces per round: at most two per lane
+constexpr int kMergeMinChunk = 8;
+constexpr int kRec16 = kPartialFloats * 4 / 16;   // 16-byte copies per record
+// shared memory per staged piece: its record and its kGroup weights
+constexpr int kMergePieceSmem = (kPartialFloats + kGroup) * 4;
+static_assert(kMergeThreads == 256 && kPartialFloats % 4 == 0, "merge layout");
 
-// Three CTAs' worth of registers per SM (at most 85 per thread, 80 used):
-// one merge CTA fits beside two one-query decode CTAs (see decode_kernel_q1).
+// Three CTAs' worth of registers per SM (at most 85 per thread): one merge
+// CTA fits beside two one-query decode CTAs (see decode_kernel_q1), and the
+// host sizes `chunk` so that its shared memory fits there too.
 // kNq: queries per sequence, 0 = read from the arguments; kTable: splits
 // from decode's table (batches above kMergeScanMaxBatch), else from the
 // lengths.
 template <int kNq, bool kBf16, bool kTable>
-__global__ void __launch_bounds__(kMergeWarps * 32, 3)
-    merge_kernel(const DecodeArgs a, int32_t decode_grid) {
-  __shared__ __align__(16) float s_part[kMergeWarps][kPartialFloats];
+__global__ void __launch_bounds__(kMergeThreads, 3)
+    merge_kernel(const DecodeArgs a, int32_t decode_grid, int32_t chunk) {
+  extern __shared__ __align__(16) float s_rec[];   // [chunk][kPartialFloats], then [chunk][kGroup]
   __shared__ int32_t s_sum[2][kMergeWarps];
+  __shared__ float s_scale[kGroup], s_inv[kGroup];
   pdl_trigger();
   const int g = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1167,8 +1085,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32, 3)
     }
     int Lb = a.seq_lens[b];
     if (Lb < 0 || Lb > cap || (Lb > 0 && Lb < a.num_queries)) Lb = 0;
-    const int64_t chunk = range_chunk(pages_all, a.batch, decode_grid, a.min_chunk);
-    const int2 sp = split_of(pages_before, b, (Lb + kTokens - 1) / kTokens, chunk);
+    const int64_t range = range_chunk(pages_all, a.batch, decode_grid, a.min_chunk);
+    const int2 sp = split_of(pages_before, b, (Lb + kTokens - 1) / kTokens, range);
     K = sp.y;
     c_first = sp.x;
     // This grid's completion is what the next programmatically dependent
@@ -1191,23 +1109,69 @@ __global__ void __launch_bounds__(kMergeWarps * 32, 3)
   if (K <= 1) return;
   const int nq = kNq > 0 ? kNq : a.num_queries;   // kNq == 0: any count
   const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + c_first;
-  const int parts = min(kMergeWarps, K);
   const OutRowsT<kBf16> out = out_rows<kBf16>(a, b, g);
-#pragma unroll
+  float* s_w = s_rec + static_cast<size_t>(chunk) * kPartialFloats;
+  const int h = threadIdx.x / kDim, d = threadIdx.x % kDim;   // this thread's output element
   for (int qi = 0; qi < nq; ++qi) {   // a piece's record of query qi: slot * nq + qi
-    if (warp < parts) {
-      const int cnt = (K - warp + kMergeWarps - 1) / kMergeWarps;
-      merge_partials<false>(a.partials + ((S0 + warp) * nq + qi) * kPartialFloats, cnt,
-                            kMergeWarps * nq, s_part[warp],
-                            static_cast<const OutRowsT<kBf16>*>(nullptr), 0, lane);
+    float M = -INFINITY, S = 0.f;     // warp h < kGroup: head h's running max and sum
+    float O = 0.f;
+    for (int c0 = 0; c0 < K; c0 += chunk) {
+      const int n = min(chunk, K - c0);
+      const float* src = a.partials + ((S0 + c0) * nq + qi) * kPartialFloats;
+      for (int i = threadIdx.x; i < n * kRec16; i += kMergeThreads) {
+        const int s = i / kRec16, o = 4 * (i - s * kRec16);
+        cp_async16(smem_addr(s_rec + s * kPartialFloats + o),
+                   src + static_cast<int64_t>(s) * nq * kPartialFloats + o);
+      }
+      cp_async_wait_all();
+      __syncthreads();
+      if (warp < kGroup) {   // head `warp`: weights of this round's pieces, rescale, sum
+        const bool has0 = lane < n, has1 = lane + 32 < n;
+        const float* r0 = s_rec + lane * kPartialFloats + warp;
+        const float* r1 = s_rec + (lane + 32) * kPartialFloats + warp;
+        const float m0 = has0 ? r0[0] : -INFINITY, m1 = has1 ? r1[0] : -INFINITY;
+        float mc = fmaxf(m0, m1);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mc = fmaxf(mc, __shfl_xor_sync(kFull, mc, off));
+        const float mn = fmaxf(M, mc);
+        // a piece whose pages were all skipped has m = -inf and weight 0
+        const float scale = (mn == -INFINITY) ? 1.f : fast_exp2(M - mn);
+        const float w0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - mn);
+        const float w1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - mn);
+        if (has0) s_w[lane * kGroup + warp] = w0;
+        if (has1) s_w[(lane + 32) * kGroup + warp] = w1;
+        float sc = fmaf(w1, has1 ? r1[kGroup] : 0.f, w0 * (has0 ? r0[kGroup] : 0.f));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sc += __shfl_xor_sync(kFull, sc, off);
+        S = fmaf(S, scale, sc);
+        M = mn;
+        if (lane == 0) s_scale[warp] = scale;
+      }
+      __syncthreads();
+      O *= s_scale[h];
+      const float* acc = s_rec + 2 * kGroup + h * kDim + d;
+#pragma unroll 4
+      for (int s = 0; s < n; ++s) O = fmaf(s_w[s * kGroup + h], acc[s * kPartialFloats], O);
+      __syncthreads();   // the next round (or query) restages s_rec, s_w and s_scale
     }
+    if (warp < kGroup && lane == 0) s_inv[warp] = S > 0.f ? 1.f / S : 0.f;
     __syncthreads();
-    if (warp == 0) merge_partials<true>(&s_part[0][0], parts, 1, nullptr, &out, qi, lane);
-    if (qi + 1 < nq) __syncthreads();   // s_part is rewritten for the next query
+    out.put(qi, h, d, O * s_inv[h]);
   }
 }
 
 // ---------------------------------------------------------------- host side --
+
+using MergeFn = void (*)(const DecodeArgs, int32_t, int32_t);
+
+// The merge kernel for (queries per sequence, BF16 output, split table).
+static MergeFn merge_fn(int nq, bool bf16, bool table) {
+  if (table)
+    return nq == 1 ? (bf16 ? merge_kernel<1, true, true> : merge_kernel<1, false, true>)
+                   : (bf16 ? merge_kernel<0, true, true> : merge_kernel<0, false, true>);
+  return nq == 1 ? (bf16 ? merge_kernel<1, true, false> : merge_kernel<1, false, false>)
+                 : (bf16 ? merge_kernel<0, true, false> : merge_kernel<0, false, false>);
+}
 
 // The kernel that runs compute type C.
 template <class C, bool kTable>
@@ -1279,7 +1243,24 @@ cudaError_t prepare_decode_kernels(int device) {
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              optin - static_cast<int>(fa.sharedSizeBytes));
     if (e != cudaSuccess) return e;
+    // all of the SM's unified memory as shared memory, for decode and merge
+    // CTAs side by side (the decode kernels read nothing through L1 that
+    // needs more than what is left)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
   }
+  for (int nq : {1, 2})
+    for (bool bf16 : {false, true})
+      for (bool table : {false, true}) {
+        const void* fn = reinterpret_cast<const void*>(merge_fn(nq, bf16, table));
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMergeMaxChunk * kMergePieceSmem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+      }
   return cudaSuccess;
 }
 
@@ -1309,6 +1290,27 @@ int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ct
   const int64_t slots = static_cast<int64_t>(kKvHeads) * (batch + plan->grid);
   plan->records_bytes = static_cast<size_t>(slots) * num_queries * kPartialFloats * sizeof(float);
   plan->ws_bytes = plan->records_bytes + static_cast<size_t>(plan->grid) * sizeof(int2);
+  // Merge rounds: as many pieces as fit in the shared memory an SM has left
+  // beside its decode CTAs (so that a merge CTA can wait there while decode
+  // runs), within [kMergeMinChunk, kMergeMaxChunk].
+  int sm_smem = 0, reserved = 0;
+  if (cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, device) !=
+          cudaSuccess)
+    return PKV_ERR_CUDA;
+  cudaFuncAttributes mfa;
+  if (cudaFuncGetAttributes(&mfa, reinterpret_cast<const void*>(merge_fn(1, false, false))) !=
+      cudaSuccess)
+    return PKV_ERR_CUDA;
+  const int64_t left = static_cast<int64_t>(sm_smem) -
+                       static_cast<int64_t>(per_sm) * (smem + fa.sharedSizeBytes + reserved) -
+                       reserved - static_cast<int64_t>(mfa.sharedSizeBytes);
+  const int64_t fit = left / kMergePieceSmem;
+  plan->merge_chunk = static_cast<int>(fit < kMergeMinChunk   ? kMergeMinChunk
+                                       : fit > kMergeMaxChunk ? kMergeMaxChunk
+                                                              : fit);
+  plan->merge_smem = static_cast<size_t>(plan->merge_chunk) * kMergePieceSmem;
   return PKV_OK;
 }
 
@@ -1337,22 +1339,17 @@ cudaError_t launch_decode(const DecodePlan& plan, const CUtensorMap& tmap, const
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kKvHeads, a.batch <= kMergeScanMaxBatch ? a.batch : plan.grid);
-  cfg.blockDim = dim3(kMergeWarps * 32);
+  cfg.blockDim = dim3(kMergeThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = (flags & kLaunchPdl) ? 1 : 0;
-  const bool table = a.batch > kMergeScanMaxBatch;
-  auto merge =
-      table ? (a.num_queries == 1
-                   ? (a.out_bf16 ? merge_kernel<1, true, true> : merge_kernel<1, false, true>)
-                   : (a.out_bf16 ? merge_kernel<0, true, true> : merge_kernel<0, false, true>))
-            : (a.num_queries == 1
-                   ? (a.out_bf16 ? merge_kernel<1, true, false> : merge_kernel<1, false, false>)
-                   : (a.out_bf16 ? merge_kernel<0, true, false> : merge_kernel<0, false, false>));
-  return cudaLaunchKernelEx(&cfg, merge, a, static_cast<int32_t>(plan.grid));
+  cfg.dynamicSmemBytes = plan.merge_smem;
+  return cudaLaunchKernelEx(&cfg, merge_fn(a.num_queries, a.out_bf16, a.batch > kMergeScanMaxBatch),
+                            a, static_cast<int32_t>(plan.grid),
+                            static_cast<int32_t>(plan.merge_chunk));
 }
 
 }  // namespace pkv

@@ -245,6 +245,8 @@ struct DecodePlan {
   size_t smem;       // dynamic shared memory bytes
   size_t records_bytes;  // workspace bytes of the partial records (at its start)
   size_t ws_bytes;   // workspace bytes: the records, then the split table [grid] int2
+  int merge_chunk;   // pieces the merge kernel stages in shared memory per round
+  size_t merge_smem;  // its dynamic shared memory bytes
 };
 
 int plan_decode(int device, int sm_count, int32_t batch, int kernel, int grid_ctas,
