@@ -702,6 +702,10 @@ __device__ __forceinline__ void flush_unit(const C& cmp, const DecodeArgs& a,
 // physical page, and (sequence << kInfoSeqShift) | kInfoRecent (one of the
 // sequence's last two pages) | kInfoLast (its last page) | kInfoStart
 // (starts a sequence in this range).
+// A range of at most kS + kShortRest pages prefetches, once its dependency
+// wait is over, all its pages beyond the stages into L2.
+constexpr int kShortRest = 4;
+
 constexpr int32_t kInfoStart = 1, kInfoLast = 2, kInfoRecent = 4;
 constexpr int kInfoSeqShift = 3;
 
@@ -890,9 +894,22 @@ __device__ __forceinline__ void decode_body(const CUtensorMap& tmap, const Decod
   for (int b = blockIdx.x * kWarps + warp; b < B; b += G * kWarps)
     if (s_pfx[b + 1] == s_pfx[b]) zero_rows(a, b, lane);
   if (n <= 0) return;
-  if (warp == 0)
+  if (warp == 0) {
     for (int r = 0; r < n && r < kS; ++r)
       issue(r, (early_mask >> r) & 1u ? kIssueRows : kIssuePage | kIssueRows);
+    // A short range spends most of its time starting up: its pages beyond
+    // the stages would each wait for a stage to free before their load even
+    // starts.  So they all go to L2 now, and the stage loads that follow hit
+    // there.  Longer ranges reach the steady state of the two-stage pipeline,
+    // where extra requests only delay other CTAs' loads (measured: prefetching
+    // ahead on every range is much slower on short-context batches).
+    if (n <= kS + kShortRest)
+      for (int r = kS; r < n; ++r) {   // r < 32: a first-batch page
+        const int32_t phys = __shfl_sync(kFull, cur_phys, r);
+        if (lane == 0 && static_cast<uint32_t>(phys) < static_cast<uint32_t>(a.num_pages))
+          bulk_prefetch_l2(a.pool + static_cast<int64_t>(phys) * (kPageBytes / 2), kPageBytes);
+      }
+  }
   // After a timed-out wait: wait (bounded) for the copies still in flight
   // into this CTA's stages, pages k0 .. issued-1, before the CTA exits.
   auto drain = [&](int k0) {
