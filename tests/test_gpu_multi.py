@@ -193,3 +193,30 @@ def test_large_batch_split_table(grid, nq, bf16):
     assert np.isfinite(got).all()
     assert max_err(got, want) <= tol
     assert not got[300].any()
+
+
+@pytest.mark.parametrize("nq", [1, 2])
+def test_merge_in_many_rounds_when_decode_leaves_little_shared_memory(nq):
+    # About 3,400 sequences: every decode CTA keeps the batch's lengths and
+    # page-count prefix in shared memory, so the shared memory an SM has left
+    # beside two decode CTAs (what the merge kernel stages its records in)
+    # holds only a few records, and the two long sequences, split over ~40
+    # CTAs each, are merged in many rounds with the running max rescaled
+    # between them.  Checked against the oracle on every sequence.
+    rng = np.random.default_rng(900 + nq)
+    lens = [int(x) for x in rng.integers(nq, 40, 3400)]
+    lens[7], lens[2000], lens[3399] = 30000, 24000, 0
+    c = make_case(lens, seed=901, spare_pages=2)
+    g = GpuCase(c)
+    q = _q2(c, 5, nq)
+    if nq == 1:
+        got = pkv.decode_general(u16_to_bf16(q[:, 0]), g.pool, g.bt, g.sl, 0, 0.125)
+        torch.cuda.synchronize()
+        got = _f64(got)[:, None]
+    else:
+        got = _f64(_run(g, q, nq))
+    assert pkv.get_device_error(g.pool) == 0
+    want = oracle.decode_multi(q, c["pool"], c["bt"], c["seq_lens"], 0, 0.125)
+    assert np.isfinite(got).all()
+    assert max_err(got, want) <= ATOL
+    assert not got[3399].any()
