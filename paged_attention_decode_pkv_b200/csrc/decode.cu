@@ -1042,18 +1042,18 @@ __global__ void __maxnreg__(kQ1Regs)
 //   S[h] = sum_s w_s[h] l_s[h],  out[h][d] = (sum_s w_s[h] acc_s[h][d]) / S[h]
 // (zero where S == 0).  The records are staged in shared memory `chunk` at a
 // time (one round for every unit of up to `chunk` pieces; a running max
-// rescales between rounds).  Thread (h, d) accumulates output element
-// (h, d); the two warps of head h each compute that head's weights (lane s
-// holds pieces s and s + 32, handed to the other lanes by shuffles) and S,
-// so a round needs no barrier beyond the one after its copies.
+// rescales between rounds).  Per round, warp h < 4 computes head h's weights
+// (lane s holds pieces s and s + 32) and the round's share of S; then each of
+// the 256 threads accumulates one output element (h, d) over the round's
+// pieces in order.
 // ---------------------------------------------------------------------------
 constexpr int kMergeThreads = kGroup * kDim;   // one output element per thread
 constexpr int kMergeWarps = kMergeThreads / 32;
 constexpr int kMergeMaxChunk = 64;             // pieces per round: at most two per lane
 constexpr int kMergeMinChunk = 8;
 constexpr int kRec16 = kPartialFloats * 4 / 16;   // 16-byte copies per record
-// shared memory per staged piece: its record
-constexpr int kMergePieceSmem = kPartialFloats * 4;
+// shared memory per staged piece: its record and its kGroup weights
+constexpr int kMergePieceSmem = (kPartialFloats + kGroup) * 4;
 static_assert(kMergeThreads == 256 && kPartialFloats % 4 == 0, "merge layout");
 
 // Three CTAs' worth of registers per SM (at most 85 per thread): one merge
@@ -1065,8 +1065,9 @@ static_assert(kMergeThreads == 256 && kPartialFloats % 4 == 0, "merge layout");
 template <int kNq, bool kBf16, bool kTable>
 __global__ void __launch_bounds__(kMergeThreads, 3)
     merge_kernel(const DecodeArgs a, int32_t decode_grid, int32_t chunk) {
-  extern __shared__ __align__(16) float s_rec[];   // [chunk][kPartialFloats]
+  extern __shared__ __align__(16) float s_rec[];   // [chunk][kPartialFloats], then [chunk][kGroup]
   __shared__ int32_t s_sum[2][kMergeWarps];
+  __shared__ float s_scale[kGroup], s_inv[kGroup];
   pdl_trigger();
   const int g = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1126,12 +1127,10 @@ __global__ void __launch_bounds__(kMergeThreads, 3)
   const int nq = kNq > 0 ? kNq : a.num_queries;   // kNq == 0: any count
   const int64_t S0 = static_cast<int64_t>(g) * (a.batch + decode_grid) + b + c_first;
   const OutRowsT<kBf16> out = out_rows<kBf16>(a, b, g);
+  float* s_w = s_rec + static_cast<size_t>(chunk) * kPartialFloats;
   const int h = threadIdx.x / kDim, d = threadIdx.x % kDim;   // this thread's output element
   for (int qi = 0; qi < nq; ++qi) {   // a piece's record of query qi: slot * nq + qi
-    // every warp keeps its head's running max and sum (the two warps of a
-    // head compute the same weights, so no barrier is needed between the
-    // weights and the accumulation)
-    float M = -INFINITY, S = 0.f;
+    float M = -INFINITY, S = 0.f;     // warp h < kGroup: head h's running max and sum
     float O = 0.f;
     for (int c0 = 0; c0 < K; c0 += chunk) {
       const int n = min(chunk, K - c0);
@@ -1143,33 +1142,38 @@ __global__ void __launch_bounds__(kMergeThreads, 3)
       }
       cp_async_wait_all();
       __syncthreads();
-      // head h's weights of this round's pieces: lane s holds pieces s, s + 32
-      const bool has0 = lane < n, has1 = lane + 32 < n;
-      const float* r0 = s_rec + lane * kPartialFloats + h;
-      const float* r1 = r0 + 32 * kPartialFloats;
-      const float m0 = has0 ? r0[0] : -INFINITY, m1 = has1 ? r1[0] : -INFINITY;
-      float mc = fmaxf(m0, m1);
+      if (warp < kGroup) {   // head `warp`: weights of this round's pieces, rescale, sum
+        const bool has0 = lane < n, has1 = lane + 32 < n;
+        const float* r0 = s_rec + lane * kPartialFloats + warp;
+        const float* r1 = s_rec + (lane + 32) * kPartialFloats + warp;
+        const float m0 = has0 ? r0[0] : -INFINITY, m1 = has1 ? r1[0] : -INFINITY;
+        float mc = fmaxf(m0, m1);
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mc = fmaxf(mc, __shfl_xor_sync(kFull, mc, off));
-      const float mn = fmaxf(M, mc);
-      // a piece whose pages were all skipped has m = -inf and weight 0
-      const float scale = (mn == -INFINITY) ? 1.f : fast_exp2(M - mn);
-      const float w0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - mn);
-      const float w1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - mn);
-      float sc = fmaf(w1, has1 ? r1[kGroup] : 0.f, w0 * (has0 ? r0[kGroup] : 0.f));
+        for (int off = 16; off > 0; off >>= 1) mc = fmaxf(mc, __shfl_xor_sync(kFull, mc, off));
+        const float mn = fmaxf(M, mc);
+        // a piece whose pages were all skipped has m = -inf and weight 0
+        const float scale = (mn == -INFINITY) ? 1.f : fast_exp2(M - mn);
+        const float w0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - mn);
+        const float w1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - mn);
+        if (has0) s_w[lane * kGroup + warp] = w0;
+        if (has1) s_w[(lane + 32) * kGroup + warp] = w1;
+        float sc = fmaf(w1, has1 ? r1[kGroup] : 0.f, w0 * (has0 ? r0[kGroup] : 0.f));
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sc += __shfl_xor_sync(kFull, sc, off);
-      S = fmaf(S, scale, sc);
-      M = mn;
-      float o = O * scale;
+        for (int off = 16; off > 0; off >>= 1) sc += __shfl_xor_sync(kFull, sc, off);
+        S = fmaf(S, scale, sc);
+        M = mn;
+        if (lane == 0) s_scale[warp] = scale;
+      }
+      __syncthreads();
+      O *= s_scale[h];
       const float* acc = s_rec + 2 * kGroup + h * kDim + d;
 #pragma unroll 4
-      for (int s = 0; s < n; ++s)
-        o = fmaf(__shfl_sync(kFull, s < 32 ? w0 : w1, s & 31), acc[s * kPartialFloats], o);
-      O = o;
-      if (c0 + chunk < K || qi + 1 < nq) __syncthreads();   // s_rec is restaged next
+      for (int s = 0; s < n; ++s) O = fmaf(s_w[s * kGroup + h], acc[s * kPartialFloats], O);
+      __syncthreads();   // the next round (or query) restages s_rec, s_w and s_scale
     }
-    out.put(qi, h, d, O * (S > 0.f ? 1.f / S : 0.f));
+    if (warp < kGroup && lane == 0) s_inv[warp] = S > 0.f ? 1.f / S : 0.f;
+    __syncthreads();
+    out.put(qi, h, d, O * s_inv[h]);
   }
 }
 
